@@ -1,0 +1,346 @@
+"""Pins of the CPU oracle to facts outside itself.
+
+Each check takes the oracle module and raises AssertionError on a mismatch.  They
+compare the oracle with exact rational arithmetic (fractions), with brute-force
+enumeration on tiny inputs, with closed forms and invariants, and with hand-derived
+fixtures.  test_oracle_pins runs them on the oracle; test_oracle_mutants plants
+plausible mistakes in the oracle and checks that some pin catches each one.
+"""
+import math
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+
+from synth import gen
+from synth.configs import QUEST_ALPHA
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+INF = float("inf")
+
+
+# --------------------------------------------------------------- exact references
+def exact_fp16_round(v):
+    """Nearest fp16 value (ties to even) of a rational, or +-inf on overflow."""
+    v = Fraction(v)
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = Fraction(2) ** (max(e, -14) - 10)
+    n = a / q
+    fl = n.numerator // n.denominator
+    r = n - fl
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    val = fl * q
+    if val > 65504:
+        return sign * INF
+    return sign * val
+
+
+def _as_float(v):
+    return float(v) if not isinstance(v, float) else v
+
+
+def bits_of_lsb_first(byts, bits):
+    """Codes from packed bytes by walking the LSB-first bit string one bit at a time."""
+    codes = []
+    n_codes = len(byts) * 8 // bits
+    for i in range(n_codes):
+        c = 0
+        for k in range(bits):
+            n = bits * i + k
+            c |= ((int(byts[n // 8]) >> (n % 8)) & 1) << k
+        codes.append(c)
+    return codes
+
+
+# ----------------------------------------------------------------------------- fp16
+def check_fp16_rounding(orc):
+    rng = np.random.default_rng(7)
+    vals = list(rng.standard_normal(300) * np.exp(rng.uniform(-25, 12, 300)))
+    # midpoints between neighbouring fp16 numbers, and one ulp of fp64 either side
+    for base in [1.0, 1.5, 3.0, 1000.0, 2.0 ** -14, 2.0 ** -20, 60000.0]:
+        h = np.float16(base)
+        nxt = np.nextafter(h, np.float16(np.inf))
+        mid = (float(h) + float(nxt)) / 2
+        vals += [mid, np.nextafter(mid, 0), np.nextafter(mid, np.inf), -mid]
+    vals += [65504.0, 65519.99, 65520.0, 70000.0, 2.0 ** -25, 2.0 ** -26, 3 * 2.0 ** -26, 0.0]
+    vals = np.array(vals, dtype=np.float64)
+    got = orc.fp16_round(vals)
+    for v, g in zip(vals, got):
+        e = exact_fp16_round(Fraction(float(v)))
+        e = e if isinstance(e, float) else float(e)
+        assert g == e, (v, g, e)
+    # the library conversion numpy float64 -> float16 is correctly rounded as well
+    with np.errstate(over="ignore"):
+        lib = vals.astype(np.float16).astype(np.float64)
+    np.testing.assert_array_equal(got, lib)
+
+
+# ------------------------------------------------------------------- QuEST grid
+def _quest_groups():
+    x = gen.fp32_groups((24, 128), seed=31).numpy().astype(np.float64)
+    # constant-magnitude group, a ramp, and a group with values exactly on thresholds
+    x[0] = np.where(np.arange(128) % 2 == 0, 0.75, -0.75)
+    x[1] = np.arange(128) - 63.5
+    return x
+
+
+def check_quest_step(orc):
+    x = _quest_groups()
+    getcontext().prec = 60
+    for bits in (2, 3, 4):
+        alpha = QUEST_ALPHA[bits]
+        got = orc.quest_meta(x, bits, alpha)
+        for gi in range(x.shape[0]):
+            s = sum(Fraction(float(v)) ** 2 for v in x[gi])
+            rms = (Decimal(s.numerator) / Decimal(s.denominator) / Decimal(128)).sqrt()
+            pre = Decimal(Fraction(alpha).numerator) / Decimal(Fraction(alpha).denominator) * rms
+            pre = Fraction(pre) * Fraction(2) ** (1 - bits)
+            assert got[gi] == _as_float(exact_fp16_round(pre)), (bits, gi)
+    # closed form: every |x| = 0.75 -> RMS = 0.75
+    for bits in (2, 3, 4):
+        d = orc.quest_meta(x[:1], bits, QUEST_ALPHA[bits])[0]
+        assert d == float(exact_fp16_round(Fraction(QUEST_ALPHA[bits]) * Fraction(3, 4)
+                                           * Fraction(2) ** (1 - bits)))
+
+
+def check_quest_codes_bruteforce(orc):
+    x = _quest_groups()
+    for bits in (2, 3, 4):
+        delta = orc.quest_meta(x, bits, QUEST_ALPHA[bits])
+        # put some values exactly on thresholds j*Delta and one fp64 ulp either side
+        xx = x.copy()
+        half = 1 << (bits - 1)
+        for gi in range(2, 10):
+            for k, j in enumerate(range(-(half - 1), half)):
+                xx[gi, 3 * k] = j * delta[gi]
+                xx[gi, 3 * k + 1] = np.nextafter(j * delta[gi], -np.inf)
+                xx[gi, 3 * k + 2] = np.nextafter(j * delta[gi], np.inf)
+        codes = orc.quest_codes(xx, delta, bits)
+        for gi in range(xx.shape[0]):
+            d = Fraction(float(delta[gi]))
+            for i in range(128):
+                v = Fraction(float(xx[gi, i]))
+                best = None
+                for c in range(1 << bits):
+                    err = abs(v - (c - half + Fraction(1, 2)) * d)
+                    if best is None or err <= best[0]:   # ties go to the upper code
+                        best = (err, c)
+                assert codes[gi, i] == best[1], (bits, gi, i, float(v), codes[gi, i], best[1])
+        deq = orc.quest_dequant(codes, delta, bits)
+        inside = (xx >= -half * delta[:, None]) & (xx < half * delta[:, None])
+        assert np.all(np.abs(xx - deq)[inside] <= (delta[:, None] / 2 + 0 * xx)[inside])
+
+
+def check_quest_degenerate(orc):
+    x = np.zeros((2, 128))
+    for bits in (2, 3, 4):
+        d = orc.quest_meta(x, bits, QUEST_ALPHA[bits])
+        assert np.all(d == 0.0)
+        assert np.all(orc.quest_codes(x, d, bits) == 1 << (bits - 1))
+        assert np.all(orc.quest_dequant(orc.quest_codes(x, d, bits), d, bits) == 0.0)
+
+
+# ---------------------------------------------------------------- percentile affine
+def check_affine_bruteforce(orc):
+    x = gen.fp32_groups((12, 128), seed=41).numpy().astype(np.float64)
+    x[0, :] = np.linspace(-3, 3, 128).astype(np.float32)
+    for bits in (2, 3, 4):
+        levels = (1 << bits) - 1
+        scale, zero = orc.affine_meta(x, bits, 2, 125)
+        xx = x.copy()
+        for gi in range(1, 6):       # values exactly on the half-way points
+            for j in range(levels):
+                t = zero[gi] + (j + 0.5) * scale[gi]
+                xx[gi, 5 + j] = np.float32(t) if float(np.float32(t)) == t else xx[gi, 5 + j]
+        codes = orc.affine_codes(xx, scale, zero, bits)
+        for gi in range(x.shape[0]):
+            srt = sorted(Fraction(float(v)) for v in x[gi])
+            lo, hi = srt[2], srt[125]
+            e_scale = exact_fp16_round((hi - lo) / levels)
+            e_zero = exact_fp16_round(lo)
+            assert scale[gi] == float(e_scale) and zero[gi] == float(e_zero), (bits, gi)
+            for i in range(128):
+                v = Fraction(float(xx[gi, i]))
+                best = None
+                for c in range(levels + 1):
+                    err = abs(v - (e_zero + c * e_scale))
+                    if best is None or err < best[0] or (err == best[0] and c % 2 == 0):
+                        best = (err, c)
+                assert codes[gi, i] == best[1], (bits, gi, i, float(v))
+        deq = orc.affine_dequant(codes, scale, zero)
+        inside = (xx >= zero[:, None]) & (xx <= (zero + levels * scale)[:, None])
+        assert np.all((np.abs(xx - deq) <= scale[:, None] / 2)[inside])
+
+
+def check_affine_degenerate(orc):
+    x = np.full((1, 128), 1.25)
+    s, z = orc.affine_meta(x, 2, 2, 125)
+    assert s[0] == 0.0 and z[0] == 1.25
+    assert np.all(orc.affine_codes(x, s, z, 2) == 0)
+    assert np.all(orc.affine_dequant(orc.affine_codes(x, s, z, 2), s, z) == 1.25)
+
+
+# ------------------------------------------------------------------------ packing
+def check_pack_golden(orc):
+    with open(os.path.join(GOLDEN, "pack_ramp.txt")) as f:
+        rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
+    for bits_s, hexs in rows:
+        bits = int(bits_s)
+        codes = (np.arange(128) % (1 << bits)).astype(np.uint8)
+        period = bytes.fromhex(hexs)
+        expect = (period * (16 * bits // len(period) + 1))[: 16 * bits]
+        got = orc.pack_codes(codes[None], bits)[0]
+        assert bytes(got.tobytes()) == expect, bits
+    rng = np.random.default_rng(3)
+    for bits in (2, 3, 4):
+        c = rng.integers(0, 1 << bits, size=(5, 128)).astype(np.uint8)
+        p = orc.pack_codes(c, bits)
+        assert p.shape == (5, 16 * bits)
+        np.testing.assert_array_equal(orc.unpack_codes(p, bits), c)
+        for r in range(5):
+            assert bits_of_lsb_first(p[r], bits) == list(c[r])
+
+
+# ---------------------------------------------------------------------- transform
+def check_transform(orc):
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal((3, 2, 2, 128)).astype(np.float32).astype(np.float64)
+    eye = np.stack([np.eye(128)] * 2)
+    np.testing.assert_array_equal(orc.transform_keys(k, eye), k)
+    t, tinv = gen.key_transform_pair(np.random.default_rng(9))
+    t32 = np.stack([t.astype(np.float32).astype(np.float64), np.eye(128)[::-1]])
+    x = orc.transform_keys(k, t32)
+    for (a, b, h) in [(0, 0, 0), (2, 1, 0), (1, 0, 1)]:
+        for i in (0, 5, 127):
+            ex = sum(Fraction(float(t32[h, i, j])) * Fraction(float(k[a, b, h, j]))
+                     for j in range(128))
+            assert abs(x[a, b, h, i] - float(ex)) <= 1e-13 * (1 + abs(float(ex))), (a, b, h, i)
+    # T_k^{-T} from the closed form is the numeric inverse-transpose; orthogonal T maps to itself
+    np.testing.assert_allclose(tinv, np.linalg.inv(t).T, atol=1e-12)
+    q = gen.haar_orthogonal(np.random.default_rng(4))
+    np.testing.assert_allclose(np.linalg.inv(q).T, q, atol=1e-12)
+    # query map: head h uses KV head h // g
+    qq = rng.standard_normal((2, 4, 128))
+    m = np.stack([t, np.eye(128)])
+    out = orc.transform_query(qq, m, 2)
+    for b in range(2):
+        for h in range(4):
+            ex = m[h // 2] @ qq[b, h]
+            np.testing.assert_allclose(out[b, h], ex, rtol=1e-12, atol=1e-12)
+
+
+def check_unquantized_invariance(orc):
+    """(T^{-T} q) . (T k) = q . k: attention with transformed queries and keys
+    equals attention on the originals."""
+    rng = np.random.default_rng(11)
+    t, tinv = gen.key_transform_pair(rng)
+    k = rng.standard_normal((1, 64, 1, 128)) * 3
+    q = rng.standard_normal((1, 4, 128))
+    x = orc.transform_keys(k, t[None])[0, :, 0, :]
+    qt = orc.transform_query(q, tinv[None], 1)[0]
+    s1 = qt @ x.T
+    s0 = q[0] @ k[0, :, 0, :].T
+    np.testing.assert_allclose(s1, s0, rtol=1e-10, atol=1e-10)
+
+
+# ----------------------------------------------------------------------- attention
+def _small_cache(orc, kind, bits, ctx=40, batch=2, hkv=2):
+    rng = np.random.default_rng(21)
+    cache = orc.empty_cache(batch, hkv, ctx + 8, kind, bits)
+    k = rng.standard_normal((batch, ctx, hkv, 128)) * np.exp(rng.standard_normal(128))
+    v = rng.standard_normal((batch, ctx, hkv, 128))
+    alpha = QUEST_ALPHA.get(bits, 2.0)
+    st = orc.quantize_append(cache, k.astype(np.float32), v.astype(np.float32),
+                             [0] * batch, kind, bits, alpha, 2, 125)
+    assert st == 0
+    return cache
+
+
+def check_decode_bruteforce(orc):
+    for kind, bits in ((0, 2), (1, 2), (0, 3), (1, 4)):
+        cache = _small_cache(orc, kind, bits)
+        rng = np.random.default_rng(23)
+        hq, hkv = 4, 2
+        q = rng.standard_normal((2, hq, 128))
+        ctx = [40, 17]
+        tau = 1 / math.sqrt(128)
+        got = orc.decode_attention(cache, q, ctx, tau, kind, bits, hkv)
+        half = 1 << (bits - 1)
+        for b in range(2):
+            for h in range(hq):
+                kv = h // (hq // hkv)
+                kh, vh = [], []
+                for side, dst in (("k", kh), ("v", vh)):
+                    for t in range(ctx[b]):
+                        codes = bits_of_lsb_first(cache[f"{side}_codes"][b, kv, t], bits)
+                        meta = [float(np.uint16(m).view(np.float16))
+                                for m in cache[f"{side}_meta"][b, kv, t]]
+                        if kind == 0:
+                            dst.append([(c - half + 0.5) * meta[0] for c in codes])
+                        else:
+                            dst.append([meta[1] + c * meta[0] for c in codes])
+                s = [tau * sum(q[b, h, i] * kh[t][i] for i in range(128)) for t in range(ctx[b])]
+                mx = max(s)
+                p = [math.exp(v - mx) for v in s]
+                den = sum(p)
+                o = [sum(p[t] * vh[t][i] for t in range(ctx[b])) / den for i in range(128)]
+                np.testing.assert_allclose(got[b, h], o, rtol=1e-10, atol=1e-10)
+
+
+def check_decode_special(orc):
+    kind, bits = 1, 2
+    cache = _small_cache(orc, kind, bits)
+    rng = np.random.default_rng(29)
+    q = rng.standard_normal((2, 4, 128))
+    tau = 1 / math.sqrt(128)
+    # ctx_len 1: output is the first dequantized value row; ctx_len 0: zeros
+    out = orc.decode_attention(cache, q, [1, 0], tau, kind, bits, 2)
+    v0 = orc.dequant_groups(orc.unpack_codes(cache["v_codes"][0, :, 0], bits),
+                            cache["v_meta"][0, :, 0], kind, bits)
+    for h in range(4):
+        np.testing.assert_allclose(out[0, h], v0[h // 2], rtol=1e-14, atol=1e-14)
+    assert np.all(out[1] == 0)
+    # identical keys: uniform weights, output is the mean of the value rows
+    c2 = {k: v.copy() for k, v in cache.items()}
+    c2["k_codes"][:] = c2["k_codes"][:, :, :1]
+    c2["k_meta"][:] = c2["k_meta"][:, :, :1]
+    out = orc.decode_attention(c2, q, [40, 17], tau, kind, bits, 2)
+    for b, n in ((0, 40), (1, 17)):
+        vh = orc.dequant_groups(orc.unpack_codes(cache["v_codes"][b, :, :n], bits),
+                                cache["v_meta"][b, :, :n], kind, bits)
+        for h in range(4):
+            np.testing.assert_allclose(out[b, h], vh[h // 2].mean(axis=0), rtol=1e-12, atol=1e-12)
+
+
+def check_append_positions(orc):
+    cache = orc.empty_cache(2, 1, 10, 0, 2)
+    x = np.ones((2, 3, 1, 128))
+    x[1] *= -2.0
+    st = orc.quantize_append(cache, x, x, [2, 8], 0, 2, 1.99)
+    assert st == 1                                   # positions 10 of sequence 1 overflow
+    assert np.all(cache["k_codes"][0, 0, 2:5] != 0) and np.all(cache["k_codes"][0, 0, :2] == 0)
+    assert np.all(cache["k_codes"][0, 0, 5:] == 0)
+    assert np.all(cache["k_meta"][1, 0, 8:10] != 0) and np.all(cache["k_meta"][1, 0, :8] == 0)
+    # all-equal positive group: Delta = fp16(1.99 * 0.5) and every code is 2 (x >= 0, x < Delta)
+    d = float(exact_fp16_round(Fraction(1.99) / 2))
+    assert orc.fp16_value(cache["k_meta"][0, 0, 2, 0]) == d
+    assert orc.unpack_codes(cache["k_codes"][0, 0, 2], 2).tolist() == [3 if 1.0 >= d else 2] * 128
+
+
+ALL_PINS = [
+    check_fp16_rounding, check_quest_step, check_quest_codes_bruteforce, check_quest_degenerate,
+    check_affine_bruteforce, check_affine_degenerate, check_pack_golden, check_transform,
+    check_unquantized_invariance, check_decode_bruteforce, check_decode_special,
+    check_append_positions,
+]
+

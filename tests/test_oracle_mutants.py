@@ -1,0 +1,156 @@
+"""Plant plausible mistakes in the CPU oracle and check that its pins catch each one.
+
+Every mutant replaces one oracle function (module attribute, so the composite
+functions pick it up) with a version carrying one typical slip: a transposed
+operand, a wrong index or divisor, a wrong tie rule, a dropped term.  The test
+passes when at least one pin fails on the mutant.
+"""
+import numpy as np
+import pytest
+
+import oracle.wushkv_oracle as orc
+from tests import pins
+
+_orig = {name: getattr(orc, name) for name in dir(orc) if callable(getattr(orc, name))}
+
+
+def _transform_keys_transposed(k, tk):
+    k = np.asarray(k, np.float64)
+    x = np.empty_like(k)
+    for h in range(tk.shape[0]):
+        x[..., h, :] = k[..., h, :] @ np.asarray(tk[h], np.float64)      # T instead of T^T
+    return x
+
+
+def _transform_query_wrong_group(q, m, hkv):
+    q = np.asarray(q, np.float64)
+    out = np.empty_like(q)
+    for h in range(q.shape[1]):
+        out[:, h, :] = q[:, h, :] @ np.asarray(m[h % hkv], np.float64).T   # h % Hkv
+    return out
+
+
+def _quest_pre_127(x, bits, alpha):
+    x = np.asarray(x, np.float64)
+    return alpha * np.sqrt(np.sum(x * x, -1) / 127) * 2.0 ** (1 - bits)
+
+
+def _quest_pre_no_sqrt(x, bits, alpha):
+    x = np.asarray(x, np.float64)
+    return alpha * (np.sum(x * x, -1) / 128) * 2.0 ** (1 - bits)
+
+
+def _quest_pre_wrong_exp(x, bits, alpha):
+    x = np.asarray(x, np.float64)
+    return alpha * np.sqrt(np.sum(x * x, -1) / 128) * 2.0 ** (-bits)
+
+
+def _quest_codes_strict(x, delta, bits):
+    x = np.asarray(x, np.float64)
+    d = np.asarray(delta, np.float64)[..., None]
+    half = 1 << (bits - 1)
+    c = np.zeros(x.shape, np.uint8)
+    for j in range(-(half - 1), half):
+        c += (x > j * d).astype(np.uint8)                                  # > instead of >=
+    return np.where(d == 0, np.uint8(half), c).astype(np.uint8)
+
+
+def _quest_dequant_no_half(codes, delta, bits):
+    return (np.asarray(codes, np.float64) - (1 << (bits - 1))) * np.asarray(delta)[..., None]
+
+
+def _affine_pre_rank_off(x, bits, rlo, rhi):
+    return _orig["affine_prerounding"](x, bits, rlo + 1, rhi - 1)
+
+
+def _affine_pre_wrong_levels(x, bits, rlo, rhi):
+    s, lo = _orig["affine_prerounding"](x, bits, rlo, rhi)
+    return s * ((1 << bits) - 1) / (1 << bits), lo                        # / 2^b
+
+
+def _affine_codes_half_up(x, scale, zero, bits):
+    x = np.asarray(x, np.float64)
+    s = np.asarray(scale, np.float64)[..., None]
+    z = np.asarray(zero, np.float64)[..., None]
+    c = np.zeros(x.shape, np.uint8)
+    for j in range((1 << bits) - 1):
+        c += (x >= z + (j + 0.5) * s).astype(np.uint8)                    # ties always up
+    return np.where(s == 0, np.uint8(0), c).astype(np.uint8)
+
+
+def _affine_dequant_no_zero(codes, scale, zero):
+    return np.asarray(codes, np.float64) * np.asarray(scale)[..., None]
+
+
+def _pack_msb(codes, bits):
+    c = np.asarray(codes, np.uint8)
+    planes = (c[..., :, None] >> np.arange(bits, dtype=np.uint8)) & 1
+    flat = planes.reshape(c.shape[:-1] + (c.shape[-1] * bits,))
+    return np.packbits(flat, axis=-1, bitorder="big")
+
+
+def _unpack_msb(p, bits):
+    p = np.asarray(p, np.uint8)
+    flat = np.unpackbits(p, axis=-1, bitorder="big")
+    planes = flat.reshape(p.shape[:-1] + (p.shape[-1] * 8 // bits, bits)).astype(np.uint8)
+    return np.sum(planes << np.arange(bits, dtype=np.uint8), -1).astype(np.uint8)
+
+
+def _fp16_truncate(x):
+    x = np.asarray(x, np.float64)
+    with np.errstate(over="ignore"):
+        h = x.astype(np.float16).astype(np.float64)
+    # one ulp toward zero where the library rounded away from zero
+    lower = np.where(np.abs(h) > np.abs(x), np.nextafter(h.astype(np.float16), np.float16(0)).astype(np.float64), h)
+    return lower
+
+
+def _decode_scale_twice(cache, q_t, ctx, tau, kind, bits, hkv):
+    return _orig["decode_attention"](cache, q_t, ctx, tau * tau * 11.3137, kind, bits, hkv)
+
+
+def _decode_unnormalized(cache, q_t, ctx, tau, kind, bits, hkv):
+    out = _orig["decode_attention"](cache, q_t, ctx, tau, kind, bits, hkv)
+    return out * np.asarray([max(int(c), 1) for c in ctx])[:, None, None] ** 0.01
+
+
+def _decode_wrong_group(cache, q_t, ctx, tau, kind, bits, hkv):
+    q = np.asarray(q_t, np.float64)
+    hq = q.shape[1]
+    perm = [(h % hkv) * (hq // hkv) + h // hkv for h in range(hq)]        # interleaved groups
+    return _orig["decode_attention"](cache, q[:, perm], ctx, tau, kind, bits, hkv)[:, np.argsort(perm)]
+
+
+MUTANTS = {
+    "transform_keys_transposed": {"transform_keys": _transform_keys_transposed},
+    "transform_query_wrong_group": {"transform_query": _transform_query_wrong_group},
+    "quest_rms_over_127": {"quest_step_prerounding": _quest_pre_127},
+    "quest_no_sqrt": {"quest_step_prerounding": _quest_pre_no_sqrt},
+    "quest_wrong_exponent": {"quest_step_prerounding": _quest_pre_wrong_exp},
+    "quest_strict_compare": {"quest_codes": _quest_codes_strict},
+    "quest_dequant_no_half": {"quest_dequant": _quest_dequant_no_half},
+    "affine_rank_off_by_one": {"affine_prerounding": _affine_pre_rank_off},
+    "affine_wrong_levels": {"affine_prerounding": _affine_pre_wrong_levels},
+    "affine_ties_up": {"affine_codes": _affine_codes_half_up},
+    "affine_dequant_no_zero": {"affine_dequant": _affine_dequant_no_zero},
+    "pack_msb_first": {"pack_codes": _pack_msb, "unpack_codes": _unpack_msb},
+    "fp16_truncate": {"fp16_round": _fp16_truncate},
+    "decode_scale_wrong": {"decode_attention": _decode_scale_twice},
+    "decode_unnormalized": {"decode_attention": _decode_unnormalized},
+    "decode_wrong_group": {"decode_attention": _decode_wrong_group},
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    for attr, fn in MUTANTS[name].items():
+        monkeypatch.setattr(orc, attr, fn)
+    failures = []
+    for check in pins.ALL_PINS:
+        try:
+            check(orc)
+        except AssertionError:
+            failures.append(check.__name__)
+        except Exception as e:  # a crash on the mutant also counts as caught
+            failures.append(f"{check.__name__}:{type(e).__name__}")
+    assert failures, f"mutant {name} passed every pin"
