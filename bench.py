@@ -1,0 +1,420 @@
+"""Benchmark of the WUSH-KV runtime hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole hot path over the Qwen3-8B-shaped decode layer
+(batch 16, 32 query / 8 KV heads, head_dim 128, context 32768, percentile-affine
+2-bit K/V): append of the step's new token per sequence (key transform, quantize,
+pack), query map by T_k^{-T}, split-K GQA decode attention over the packed cache.
+`value` is the step's algorithmic HBM bytes / device time (GB/s); the quantize-
+append throughput is measured beside it on a 2048-token chunk (QuEST 2-bit, the
+bit-width sweep's shape).  With N > 1 (torchrun) every rank runs the same workload
+on its own GPU (independent replicas, no collective on the data path); the time is
+the max over ranks and `value` sums all ranks' bytes.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of the
+method here) on a bounded sample of the same workload on the host cores.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import gen  # noqa: E402
+from synth.configs import QWEN8B_DECODE, QWEN8B_SWEEP  # noqa: E402
+
+METRIC = "2-bit KV decode-attn HBM GB/s (% of peak) & quant-append tokens/s, 1×B200"
+TAU = 1.0 / math.sqrt(128)
+L2_FLUSH_BYTES = 512 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------- byte counts
+def group_bytes(qspec):
+    return 16 * qspec.bits + 2 * qspec.meta_per_group
+
+
+def decode_bytes(w, ctx_per_seq):
+    """Cache read (codes + meta of K and V) plus q' in and out written."""
+    cache = sum(ctx_per_seq) * w.num_kv_heads * 2 * group_bytes(w.quant)
+    return cache + w.batch * w.num_q_heads * 128 * (4 + 4)
+
+
+def append_bytes(w, n_tokens):
+    """bf16 K and V read, codes + meta written, T_k read once per KV head."""
+    return (w.batch * n_tokens * w.num_kv_heads * (2 * 256 + 2 * group_bytes(w.quant))
+            + w.num_kv_heads * 128 * 128 * 4)
+
+
+def query_bytes(w):
+    return w.batch * w.num_q_heads * 128 * (2 + 4) + w.num_kv_heads * 128 * 128 * 4
+
+
+# ------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([s.strip() for s in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows if len(r) > 8 for i in range(4)
+                          if r[5 + i].lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    if n_gpus <= 1 and "WORLD_SIZE" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(n_gpus)))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our kernels
+def build_history(dq, w, cache, tk, device):
+    """Untimed appends of positions 0 .. history-1 (chunks of 4096 tokens)."""
+    chunk = 4096
+    t = 0
+    while t < w.history:
+        n = min(chunk, w.history - t)
+        k = gen.keys(w, 0, w.batch, t, n, device=device)
+        v = gen.values(w, 0, w.batch, t, n, device=device)
+        sp = torch.full((w.batch,), t, dtype=torch.int32, device=device)
+        dq.quantize_append(cache, k, v, sp, tk)
+        t += n
+    torch.cuda.synchronize()
+
+
+def run_ours(args, rank, world, local):
+    import decode_attention_quant_b200 as dq
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = QWEN8B_DECODE
+    qs = w.quant
+    tk_np, tinv_np = gen.transforms(w)
+    tk = torch.from_numpy(tk_np).to(device)
+    tinv = torch.from_numpy(tinv_np).to(device)
+    cache = dq.PackedCache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, qs.clip_alpha, qs.rank_lo,
+                           qs.rank_hi, device=device)
+    build_history(dq, w, cache, tk, device)
+    pos = w.history                                        # the step's token goes to position ctx-1
+    k_new = gen.keys(w, 0, w.batch, pos, 1, device=device, salt=1)
+    v_new = gen.values(w, 0, w.batch, pos, 1, device=device, salt=1)
+    q = gen.queries(w, device=device).contiguous()
+    start = torch.full((w.batch,), pos, dtype=torch.int32, device=device)
+    ctx = torch.full((w.batch,), w.ctx, dtype=torch.int32, device=device)
+    q_t = torch.empty(q.shape, dtype=torch.float32, device=device)
+    out = torch.empty_like(q_t)
+    ws = torch.empty(dq.decode_workspace_bytes(cache, w.num_q_heads), dtype=torch.uint8, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        dq.quantize_append(cache, k_new, v_new, start, tk, status)
+        dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
+        dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+
+    launches_per_step = 2 + 1 + 2
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            dq.quantize_append(cache, k_new, v_new, start, tk, status)
+            ev[i][1].record(stream)
+            dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
+            ev[i][2].record(stream)
+            dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+            ev[i][3].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world)
+    ms_step = ms_total / args.steps
+    dec_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps))
+    step_bytes = decode_bytes(w, [w.ctx] * w.batch) + append_bytes(w, 1) + query_bytes(w)
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    dec_alg = decode_bytes(w, [w.ctx] * w.batch)
+    achieved = dec_alg / (dec_ms * 1e-3) / 1e9
+
+    # end to end through the C ABI with host buffers: new K/V and q in, output out
+    h_k = k_new.cpu().pin_memory()
+    h_v = v_new.cpu().pin_memory()
+    h_q = q.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    d_k, d_v, d_q = torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(q)
+
+    def e2e_step():
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        dq.quantize_append(cache, d_k, d_v, start, tk, status)
+        dq.transform_query(d_q, tinv, w.num_kv_heads, out=q_t)
+        dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    h2d = (k_new.numel() + v_new.numel() + q.numel()) * 2
+    d2h = out.numel() * 4
+
+    # quantize-append throughput: 2048-token chunk per sequence, QuEST 2-bit
+    app = bench_append(dq, device, args, world)
+    st = int(status.item())
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8 codes / fp16 meta / fp32 accumulate", "data": "synthetic",
+        "config": {"workload": f"{w.name}: 1-token append + query map + split-K decode per step",
+                   "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+                   "head_dim": 128, "ctx": w.ctx, "quantizer": "percentile-affine 2-bit ranks 2/125",
+                   "l2": "inputs larger than L2 (packed cache 302 MB > 126 MB L2)", "parallelism": f"replicas x{world}"},
+        "step_bytes": step_bytes,
+        "roofline": {"bound": "hbm", "kernel": "decode (split-K + combine)", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "alg_bytes_per_launch": dec_alg, "launch_ms": round(dec_ms, 5)},
+        "append": app,
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "device_status": st,
+    }
+    return res
+
+
+def bench_append(dq, device, args, world):
+    w = QWEN8B_SWEEP(2)
+    qs = w.quant
+    tk = torch.from_numpy(gen.transforms(w)[0]).to(device)
+    n = w.append_tokens
+    cache = dq.PackedCache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, qs.clip_alpha, device=device)
+    k = gen.keys(w, 0, w.batch, w.history, n, device=device)
+    v = gen.values(w, 0, w.batch, w.history, n, device=device)
+    sp = torch.full((w.batch,), w.history, dtype=torch.int32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for _ in range(max(3, args.warmup)):
+        dq.quantize_append(cache, k, v, sp, tk)
+    torch.cuda.synchronize()
+    times = []
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(5, args.steps)):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dq.quantize_append(cache, k, v, sp, tk)
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = max_over_ranks(statistics.median(times), world)
+    by = append_bytes(w, n)
+    peak, _ = _peaks()
+    gbs = by / (ms * 1e-3) / 1e9
+    return {"workload": f"{w.name}: 2048-token chunk x 16 sequences x 8 KV heads", "tokens_per_s":
+            round(world * w.batch * n / (ms * 1e-3), 1), "ms": round(ms, 5), "GB/s": round(world * gbs, 1),
+            "frac_of_peak": round(gbs / peak, 4), "alg_bytes": by, "l2": "flushed (512 MB write) before each rep"}
+
+
+# ------------------------------------------------------------------- oracle arm
+def oracle_sample(w, pairs, seed=0):
+    """Inputs for the oracle on `pairs` (sequence, KV head) pairs of the workload: a
+    random packed cache of the full context, the step's new token, queries."""
+    c = gen.random_cache(1, pairs, w.ctx, w.quant.kind, w.quant.bits, seed=seed)
+    c = {k: v.numpy() for k, v in c.items()}
+    for k in ("k_meta", "v_meta"):
+        c[k] = c[k].view(np.uint16)
+    tk, tinv = gen.transforms(w)
+    g = w.group
+    k_new = gen.keys(w, 0, 1, w.ctx - 1, 1).float().numpy()[:, :, :1].repeat(pairs, axis=2).astype(np.float64)
+    v_new = gen.values(w, 0, 1, w.ctx - 1, 1).float().numpy()[:, :, :1].repeat(pairs, axis=2).astype(np.float64)
+    q = gen.queries(w).float().numpy()[:1, :pairs * g].astype(np.float64)
+    return c, k_new, v_new, q, np.stack([tk[0]] * pairs), np.stack([tinv[0]] * pairs)
+
+
+def time_oracle(w, pairs, seconds_cap=30.0):
+    """One bounded oracle pass: append of 1 token, query map, decode for `pairs` pairs."""
+    sys.path.insert(0, ROOT)
+    import oracle.wushkv_oracle as orc
+    c, k_new, v_new, q, tk, tinv = oracle_sample(w, pairs)
+    qs = w.quant
+    t0 = time.perf_counter()
+    orc.quantize_append(c, k_new, v_new, [w.ctx - 1], qs.kind, qs.bits, qs.clip_alpha, qs.rank_lo, qs.rank_hi,
+                        tk=tk.astype(np.float64))
+    qt = orc.transform_query(q, tinv.astype(np.float64), pairs)
+    orc.decode_attention(c, qt, [w.ctx], TAU, qs.kind, qs.bits, pairs)
+    dt = time.perf_counter() - t0
+    # the same byte accounting as the GPU step, for the sampled pairs
+    frac = pairs / (w.batch * w.num_kv_heads)
+    by = frac * (decode_bytes(w, [w.ctx] * w.batch) + append_bytes(w, 1) + query_bytes(w))
+    return dt, by
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, pairs=32):
+    dt, by = time_oracle(w, pairs)
+    return {"value": round(by / dt / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{pairs} of {w.batch * w.num_kv_heads} (sequence, KV head) pairs at ctx {w.ctx}: "
+                      f"1-token append + query map + decode, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = QWEN8B_DECODE
+    pairs = 1
+    for _ in range(args.warmup):
+        time_oracle(w, pairs)
+    tot_t = tot_b = 0.0
+    for _ in range(args.steps):
+        dt, by = time_oracle(w, pairs)
+        tot_t += dt
+        tot_b += by
+    val = tot_b / tot_t / 1e9
+    ms = tot_t / args.steps * 1e3
+    cb = {"value": round(val, 4), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
+          "sample": f"each step: {pairs} of {w.batch * w.num_kv_heads} (sequence, KV head) pairs at ctx {w.ctx}"}
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{w.name}: 1-token append + query map + split-K decode per step (sampled)",
+                       "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+                       "ctx": w.ctx},
+            "cpu_baseline": cb, "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_ours(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(QWEN8B_DECODE)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

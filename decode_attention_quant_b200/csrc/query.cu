@@ -1,0 +1,80 @@
+// Decode-query map q' = T_k^{-T} q per query head, with T_k of the head's KV group.
+//
+// Keys are cached in the transformed basis x = T_k k (WUSH-KV: the key transform is
+// applied online after RoPE, ai4snews summary paragraph 5), so scores are kept
+// exact by mapping the query with the inverse-transpose: (T^{-T} q) . (T k) = q . k.
+// One CTA = one KV head and up to kBatchPerCta sequences; thread i owns output
+// channel i and keeps row i of T_k^{-T} in registers.
+#include "wushkv_common.cuh"
+#include "wushkv_launch.h"
+
+namespace wushkv {
+namespace {
+
+constexpr int kBatchPerCta = 4;
+
+template <bool BF16_IN>
+__global__ void __launch_bounds__(kHeadDim) transform_query_kernel(
+    const void* __restrict__ q, int batch, int hq, int hkv, const float* __restrict__ m,
+    float* __restrict__ out) {
+  extern __shared__ __align__(16) float qs[];   // [kBatchPerCta * g][128]
+  const int kv = blockIdx.x, b0 = blockIdx.y * kBatchPerCta, i = threadIdx.x;
+  const int g = hq / hkv;
+  const int nb = min(kBatchPerCta, batch - b0);
+  for (int e = i; e < nb * g * kHeadDim; e += kHeadDim) {
+    const int r = e / kHeadDim, c = e % kHeadDim;
+    const int b = b0 + r / g, h = kv * g + r % g;
+    const size_t off = ((size_t)b * hq + h) * kHeadDim + c;
+    qs[e] = BF16_IN ? __bfloat162float(static_cast<const __nv_bfloat16*>(q)[off])
+                    : static_cast<const float*>(q)[off];
+  }
+  float mr[kHeadDim];
+  const float4* mrow = reinterpret_cast<const float4*>(m + ((size_t)kv * kHeadDim + i) * kHeadDim);
+#pragma unroll
+  for (int j = 0; j < kHeadDim / 4; ++j) {
+    const float4 v = __ldg(mrow + j);
+    mr[4 * j] = v.x; mr[4 * j + 1] = v.y; mr[4 * j + 2] = v.z; mr[4 * j + 3] = v.w;
+  }
+  __syncthreads();
+#pragma unroll 1
+  for (int r = 0; r < nb * g; ++r) {
+    const float4* qr = reinterpret_cast<const float4*>(qs + r * kHeadDim);
+    float acc = 0.f;
+#pragma unroll
+    for (int j = 0; j < kHeadDim / 4; ++j) {
+      const float4 v = qr[j];
+      acc = fmaf(mr[4 * j], v.x, acc);
+      acc = fmaf(mr[4 * j + 1], v.y, acc);
+      acc = fmaf(mr[4 * j + 2], v.z, acc);
+      acc = fmaf(mr[4 * j + 3], v.w, acc);
+    }
+    const int b = b0 + r / g, h = kv * g + r % g;
+    out[((size_t)b * hq + h) * kHeadDim + i] = acc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_transform_query(const void* q, int q_dtype, int batch, int num_q_heads,
+                                   int num_kv_heads, const float* Tk_invT, float* q_out,
+                                   cudaStream_t stream) {
+  const int g = num_q_heads / num_kv_heads;
+  const int smem = kBatchPerCta * g * kHeadDim * (int)sizeof(float);
+  dim3 grid(num_kv_heads, (batch + kBatchPerCta - 1) / kBatchPerCta);
+  if (q_dtype == WUSHKV_BF16) {
+    cudaError_t e = cudaFuncSetAttribute(transform_query_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    transform_query_kernel<true><<<grid, kHeadDim, smem, stream>>>(q, batch, num_q_heads,
+                                                                   num_kv_heads, Tk_invT, q_out);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(transform_query_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    transform_query_kernel<false><<<grid, kHeadDim, smem, stream>>>(q, batch, num_q_heads,
+                                                                    num_kv_heads, Tk_invT, q_out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace wushkv

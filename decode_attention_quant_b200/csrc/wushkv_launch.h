@@ -1,0 +1,28 @@
+// Internal launcher interface between the C ABI (abi.cu) and the kernel files.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/wushkv.h"
+
+namespace wushkv {
+
+cudaError_t launch_quantize_append(const wushkv_cache& c, const void* k_new, const void* v_new,
+                                   int in_dtype, int n_new, const int32_t* start_pos,
+                                   const float* Tk, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_transform_query(const void* q, int q_dtype, int batch, int num_q_heads,
+                                   int num_kv_heads, const float* Tk_invT, float* q_out,
+                                   cudaStream_t stream);
+
+// Split count used when the caller passes num_splits = 0.
+int auto_num_splits(const wushkv_cache& c, int num_q_heads);
+size_t decode_workspace_bytes(const wushkv_cache& c, int num_q_heads, int num_splits);
+
+cudaError_t launch_decode_attention(const wushkv_cache& c, const float* q_t, int num_q_heads,
+                                    const int32_t* ctx_len, float softmax_scale, float* out,
+                                    void* workspace, int num_splits, int32_t* status,
+                                    cudaStream_t stream);
+
+}  // namespace wushkv

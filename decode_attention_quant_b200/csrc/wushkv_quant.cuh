@@ -1,0 +1,191 @@
+// Per-group clipped quantizers of WUSH-KV, one 128-value group per thread.
+//
+// QuEST-INT-style symmetric grid and OSCAR-style percentile-clipped affine grid
+// (ai4snews summary "WUSH-KV cuts 2-bit KV-cache perplexity ...", paragraphs 3-5;
+// arXiv abstract).  The grids, as this library reads them:
+//   QuEST: Delta = fp16(alpha * sqrt(sum x^2 / 128) * 2^(1-b)),
+//          code = clamp(floor(x / Delta) + 2^(b-1), 0, 2^b - 1)
+//   affine: lo, hi = values of ascending rank r_lo, r_hi; scale = fp16((hi-lo)/(2^b-1)),
+//          zero = fp16(lo), code = clamp(rne((x - zero) / scale), 0, 2^b - 1)
+// Codes must equal the exact-arithmetic decision for the given fp32 value x, so
+// every fast step carries a bracket and falls back to exact comparisons when the
+// bracket does not settle the answer:
+//   * sum of squares: fp32 chains of 16 terms (relative error < 17 * 2^-24);
+//     if fp16(pre * (1 -+ 1e-6)) disagree, the group's sum is redone in fp64.
+//   * codes: the quotient is evaluated with the reciprocal widened by 2^-20 on both
+//     sides; where the two roundings differ the group's codes are recomputed by
+//     exact threshold comparisons (fp32 for QuEST, fp64 for affine thresholds).
+#pragma once
+#include "wushkv_common.cuh"
+
+namespace wushkv {
+
+constexpr float kMagic = 12582912.0f;       // 1.5 * 2^23: integers live in the low mantissa bits
+constexpr int32_t kMagicBits = 0x4B400000;
+constexpr float kWidenDn = 0.999999046325683594f;  // 1 - 2^-20 (exact in fp32)
+constexpr float kWidenUp = 1.00000095367431641f;   // 1 + 2^-20 (exact in fp32)
+constexpr double kStepMargin = 1.0e-6;
+
+template <int BITS>
+__device__ __forceinline__ void put_code(uint32_t (&w)[4 * BITS], int i, uint32_t c) {
+  const int o = BITS * i;
+  const int wi = o >> 5;
+  const int sh = o & 31;
+  w[wi] |= c << sh;
+  if (sh + BITS > 32) w[wi + 1] |= c >> (32 - sh);
+}
+
+template <int BITS>
+__device__ __forceinline__ void clear_words(uint32_t (&w)[4 * BITS]) {
+#pragma unroll
+  for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
+}
+
+// alpha * RMS * 2^(1-b) in fp64 from a sum of squares (same operation order as the
+// plain definition: sqrt of the mean, times alpha, times a power of two).
+__device__ __forceinline__ double quest_pre(double sumsq, double alpha, int bits) {
+  const double rms = sqrt(sumsq * (1.0 / 128.0));
+  return alpha * rms * ldexp(1.0, 1 - bits);
+}
+
+// ---------------------------------------------------------------------------- QuEST
+template <int BITS>
+__device__ __forceinline__ void quest_quantize(const float (&x)[kHeadDim], double alpha,
+                                               uint32_t (&w)[4 * BITS], uint16_t& delta_bits,
+                                               int32_t& flags) {
+  constexpr int kHalf = 1 << (BITS - 1);
+  constexpr int kMaxCode = (1 << BITS) - 1;
+  float s[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) s[k] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHeadDim; ++i) s[i & 7] = fmaf(x[i], x[i], s[i & 7]);
+  const double sum_fast = (((double)s[0] + (double)s[1]) + ((double)s[2] + (double)s[3])) +
+                          (((double)s[4] + (double)s[5]) + ((double)s[6] + (double)s[7]));
+  if (!isfinite(sum_fast)) flags |= WUSHKV_STATUS_NONFINITE;
+  const double pre_fast = quest_pre(sum_fast, alpha, BITS);
+  uint16_t h = f64_to_f16_bits(pre_fast * (1.0 - kStepMargin));
+  if (h != f64_to_f16_bits(pre_fast * (1.0 + kStepMargin))) {
+    double sum = 0.0;
+#pragma unroll
+    for (int i = 0; i < kHeadDim; ++i) sum = fma((double)x[i], (double)x[i], sum);
+    h = f64_to_f16_bits(quest_pre(sum, alpha, BITS));
+  }
+  delta_bits = h;
+  const float delta = f16_bits_to_f32(h);
+  if (isinf(delta)) flags |= WUSHKV_STATUS_META_OVERFLOW;
+  clear_words<BITS>(w);
+  if (delta == 0.f) {
+#pragma unroll
+    for (int i = 0; i < kHeadDim; ++i) put_code<BITS>(w, i, kHalf);
+    return;
+  }
+  const float inv = __frcp_rn(delta);
+  const float inv_dn = __fmul_rd(inv, kWidenDn);
+  const float inv_up = __fmul_ru(inv, kWidenUp);
+  const float m = kMagic + (float)kHalf;
+  uint32_t mism = 0u;
+#pragma unroll
+  for (int i = 0; i < kHeadDim; ++i) {
+    const float y1 = __fmaf_rd(x[i], inv_dn, m);
+    const float y2 = __fmaf_rd(x[i], inv_up, m);
+    mism |= f2u(y1) ^ f2u(y2);
+    const int32_t c = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
+    put_code<BITS>(w, i, (uint32_t)c);
+  }
+  if (mism != 0u) {  // exact: count the thresholds j*Delta (exact in fp32) that x reaches
+    clear_words<BITS>(w);
+#pragma unroll
+    for (int i = 0; i < kHeadDim; ++i) {
+      uint32_t c = 0;
+#pragma unroll
+      for (int j = -(kHalf - 1); j < kHalf; ++j) c += (x[i] >= (float)j * delta) ? 1u : 0u;
+      put_code<BITS>(w, i, c);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ percentile affine
+// Smallest KSEL and largest KSEL values of the group, ascending / descending.
+template <int KSEL>
+__device__ __forceinline__ void select_extremes(const float (&x)[kHeadDim], float (&lo)[KSEL],
+                                                float (&hi)[KSEL]) {
+#pragma unroll
+  for (int k = 0; k < KSEL; ++k) {
+    lo[k] = __int_as_float(0x7f800000);
+    hi[k] = __int_as_float(0xff800000);
+  }
+#pragma unroll
+  for (int i = 0; i < kHeadDim; ++i) {
+    const float v = x[i];
+#pragma unroll
+    for (int k = KSEL - 1; k >= 1; --k) {
+      lo[k] = fminf(lo[k], fmaxf(lo[k - 1], v));
+      hi[k] = fmaxf(hi[k], fminf(hi[k - 1], v));
+    }
+    lo[0] = fminf(lo[0], v);
+    hi[0] = fmaxf(hi[0], v);
+  }
+}
+
+template <int KSEL>
+__device__ __forceinline__ float pick(const float (&a)[KSEL], int idx) {
+  float r = a[0];
+#pragma unroll
+  for (int k = 1; k < KSEL; ++k) r = (idx == k) ? a[k] : r;
+  return r;
+}
+
+template <int BITS, int KSEL>
+__device__ __forceinline__ void affine_quantize(const float (&x)[kHeadDim], int rank_lo,
+                                                int rank_hi, uint32_t (&w)[4 * BITS],
+                                                uint16_t& scale_bits, uint16_t& zero_bits,
+                                                int32_t& flags) {
+  constexpr int kMaxCode = (1 << BITS) - 1;
+  float lo_k[KSEL], hi_k[KSEL];
+  select_extremes<KSEL>(x, lo_k, hi_k);
+  float fsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHeadDim; ++i) fsum += x[i];
+  if (!isfinite(fsum)) flags |= WUSHKV_STATUS_NONFINITE;
+  const float lo = pick<KSEL>(lo_k, rank_lo);
+  const float hi = pick<KSEL>(hi_k, kHeadDim - 1 - rank_hi);
+  const double scale_pre = ((double)hi - (double)lo) / (double)kMaxCode;
+  scale_bits = f64_to_f16_bits(scale_pre);
+  zero_bits = f32_to_f16_bits(lo);
+  const float sc = f16_bits_to_f32(scale_bits);
+  const float z = f16_bits_to_f32(zero_bits);
+  if (isinf(sc) || isinf(z)) flags |= WUSHKV_STATUS_META_OVERFLOW;
+  clear_words<BITS>(w);
+  if (sc == 0.f) return;  // all codes 0: x_hat = zero
+  const float inv = __frcp_rn(sc);
+  const float inv_dn = __fmul_rd(inv, kWidenDn);
+  const float inv_up = __fmul_ru(inv, kWidenUp);
+  uint32_t mism = 0u;
+#pragma unroll
+  for (int i = 0; i < kHeadDim; ++i) {
+    const float d = __fsub_rn(x[i], z);
+    const float y1 = __fmaf_rn(d, inv_dn, kMagic);
+    const float y2 = __fmaf_rn(d, inv_up, kMagic);
+    mism |= f2u(y1) ^ f2u(y2);
+    const int32_t c = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
+    put_code<BITS>(w, i, (uint32_t)c);
+  }
+  if (mism != 0u) {  // exact: thresholds zero + (j + 1/2) scale are exact in fp64
+    clear_words<BITS>(w);
+    const double zd = (double)z, sd = (double)sc;
+#pragma unroll
+    for (int i = 0; i < kHeadDim; ++i) {
+      const double xd = (double)x[i];
+      uint32_t c = 0;
+#pragma unroll
+      for (int j = 0; j < kMaxCode; ++j) {
+        const double t = zd + ((double)j + 0.5) * sd;
+        c += (xd > t || (xd == t && (j & 1))) ? 1u : 0u;
+      }
+      put_code<BITS>(w, i, c);
+    }
+  }
+}
+
+}  // namespace wushkv

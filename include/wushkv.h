@@ -1,0 +1,176 @@
+/*
+ * wushkv.h - C ABI of the WUSH-KV runtime hot path on one NVIDIA B200 (sm_100a).
+ *
+ * The method: WUSH-KV (preprint "WUSH-KV: KV Cache Quantization with
+ * Data-Adaptive Transforms").  Its only published description here is a set of
+ * summary pages; the passages each call follows are named below as
+ *   [ai4s N]  ai4snews summary "WUSH-KV cuts 2-bit KV-cache perplexity from
+ *             OSCAR's 13.74 to 10.51 ...", paragraph N (1-6),
+ *   [blog]    cere-bro page "WUSH-KV: 2-bit KV-Cache Quantization with
+ *             Data-Adaptive Transforms" (TL;DR, flowchart, Gaps),
+ *   [abs]     the arXiv abstract as listed by readsearch.ai and searcharxiv.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless a parameter says otherwise.  All
+ *     buffers are owned by the caller; the library never allocates, frees or
+ *     synchronizes.  Every call enqueues work on `stream` (a cudaStream_t, or
+ *     NULL for the legacy default stream) and returns immediately.
+ *   - head_dim is 128 and one quantization group is one (token, KV head) row of
+ *     128 values.
+ *   - Return value: WUSHKV_OK, or a negative wushkv_error.  Argument errors are
+ *     detected on the host before anything is enqueued.  Problems only visible
+ *     on the device (see WUSHKV_STATUS_*) are OR-ed into the optional `status`
+ *     int32 (device memory, caller clears it); no kernel ever traps.
+ *   - Calls keep no state between them and are safe to issue from several
+ *     host threads on different streams.
+ */
+#ifndef WUSHKV_H_
+#define WUSHKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WUSHKV_API __attribute__((visibility("default")))
+#else
+#define WUSHKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WUSHKV_HEAD_DIM 128
+
+typedef enum {
+  WUSHKV_OK = 0,
+  WUSHKV_ERR_INVALID = -1,      /* null pointer, non-positive size, bad rank pair, ... */
+  WUSHKV_ERR_UNSUPPORTED = -2,  /* bits not in {2,3,4}, unknown kind/dtype, head_dim != 128 */
+  WUSHKV_ERR_MISALIGNED = -3,   /* a pointer is not 16-byte aligned */
+  WUSHKV_ERR_WORKSPACE = -4,    /* workspace smaller than wushkv_decode_workspace_bytes() */
+  WUSHKV_ERR_CUDA = -5          /* a CUDA runtime call or kernel launch failed */
+} wushkv_error;
+
+/* Device-side conditions, OR-ed into *status (never a trap). */
+#define WUSHKV_STATUS_CAPACITY 1       /* start_pos[b] + t >= capacity: that row was not written */
+#define WUSHKV_STATUS_NONFINITE 2      /* a group had a NaN/Inf input: its codes are unspecified */
+#define WUSHKV_STATUS_META_OVERFLOW 4  /* a step/scale/zero overflowed fp16 (stored as Inf) */
+#define WUSHKV_STATUS_CTX_OVERFLOW 8   /* ctx_len[b] > capacity: clamped to capacity */
+#define WUSHKV_STATUS_TIMEOUT 16       /* an internal pipeline wait gave up; output unspecified */
+
+/* Quantizer family [ai4s 3-5], [abs]:
+ *  QUEST_INT  - QuEST-INT-style symmetric RMS-clipped grid (the quantizer of the
+ *               pages' theory and perplexity runs).  Per group:
+ *               Delta = fp16(clip_alpha * RMS * 2^(1-bits)), RMS = sqrt(sum x^2 / 128);
+ *               code = clamp(floor(x / Delta) + 2^(bits-1), 0, 2^bits - 1);
+ *               x_hat = (code - 2^(bits-1) + 1/2) * Delta.  One fp16 meta value (Delta).
+ *  PCT_AFFINE - OSCAR-style percentile-clipped affine grid (the quantizer of the
+ *               SGLang runs).  lo, hi = elements of 0-based ascending rank
+ *               rank_lo, rank_hi; scale = fp16((hi - lo) / (2^bits - 1));
+ *               zero = fp16(lo); code = clamp(round_half_even((x - zero) / scale),
+ *               0, 2^bits - 1); x_hat = zero + code * scale.  Two fp16 meta values
+ *               (scale, zero), in that order.
+ * fp16 conversions round to nearest even once; codes are decided by exact
+ * comparisons with the grid's thresholds.  Delta == 0 gives code 2^(bits-1);
+ * scale == 0 gives code 0. */
+typedef enum { WUSHKV_QUEST_INT = 0, WUSHKV_PCT_AFFINE = 1 } wushkv_quant_kind;
+
+typedef enum { WUSHKV_BF16 = 0, WUSHKV_FP32 = 1 } wushkv_dtype;
+
+typedef struct {
+  int32_t kind;        /* wushkv_quant_kind */
+  int32_t bits;        /* 2, 3 or 4 */
+  double clip_alpha;   /* QUEST_INT clip multiplier (e.g. 1.99 / 2.34 / 2.68 for 2 / 3 / 4 bits); > 0 */
+  int32_t rank_lo;     /* PCT_AFFINE ranks; supported: 0 <= rank_lo <= 2, 125 <= rank_hi <= 127 */
+  int32_t rank_hi;
+} wushkv_quant_params;
+
+/* The packed KV cache of one layer (host struct describing caller-owned device memory).
+ *   k_codes, v_codes: uint8 [batch][num_kv_heads][capacity][16*bits].  Row
+ *       (b, h, t) is the LSB-first bit string of the group's 128 codes: code i at
+ *       bits [bits*i, bits*i + bits), bit n is bit (n mod 8) of byte n / 8.
+ *   k_meta, v_meta: fp16 bit patterns [batch][num_kv_heads][capacity][m], m = 1
+ *       (Delta) for QUEST_INT, m = 2 (scale, zero) for PCT_AFFINE.
+ *   Keys are stored in the transformed basis x = T_k k [ai4s 5]; values are stored
+ *   as given, since their transform is folded into the model weights [ai4s 5],
+ *   [blog flowchart].  Code pointers must be 16-byte aligned, meta pointers
+ *   4-byte aligned. */
+typedef struct {
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint16_t* k_meta;
+  uint16_t* v_meta;
+  int32_t batch;
+  int32_t num_kv_heads;
+  int32_t capacity;    /* T_max, tokens per sequence */
+  int32_t head_dim;    /* must be 128 */
+  wushkv_quant_params qp;
+} wushkv_cache;
+
+/* Key transform + clipped quantization + bit-packing + append.
+ * [ai4s 1]: one key transform per KV head; [ai4s 5], [blog TL;DR], [abs]: it is
+ * applied to post-RoPE keys online; keys and values are then quantized per token
+ * with a clipped quantizer and written to the cache.
+ *   k_new, v_new : [batch][n_new][num_kv_heads][128], dtype in_dtype, contiguous,
+ *                  16-byte aligned.  k_new must already be post-RoPE.
+ *   n_new        : tokens per sequence in this call (>= 1).
+ *   start_pos    : int32 [batch] (device); row t of sequence b goes to position
+ *                  start_pos[b] + t.  Positions >= capacity are skipped
+ *                  (WUSHKV_STATUS_CAPACITY).  Not modified.
+ *   Tk           : fp32 [num_kv_heads][128][128] row-major, x_i = sum_j Tk[h][i][j] k_j;
+ *                  NULL means identity (the keys are taken as already transformed,
+ *                  which is how the quantizer is tested on exact fp32 inputs).
+ *   status       : optional int32 (device).
+ * The transform runs on the tensor cores with Tk split exactly into three bf16
+ * parts (products exact, fp32 accumulation); the quantizer works on the fp32
+ * result.  Values never pass through the transform. */
+WUSHKV_API int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const void* v_new,
+                           int32_t in_dtype, int32_t n_new, const int32_t* start_pos,
+                           const float* Tk, int32_t* status, void* stream);
+
+/* Decode-query map q' = T_k^{-T} q, with T_k of the query head's KV head h / g,
+ * g = num_q_heads / num_kv_heads.  Needed because keys are cached as T_k k, and
+ * (T_k^{-T} q) . (T_k k) = q . k keeps the attention scores unchanged (implied by
+ * [ai4s 5]: keys are transformed online after RoPE while attention stays exact).
+ *   q       : [batch][num_q_heads][128], dtype q_dtype, contiguous, 16-byte aligned.
+ *   Tk_invT : fp32 [num_kv_heads][128][128] row-major (the caller computes the
+ *             inverse-transpose once per layer, off the hot path).
+ *   q_out   : fp32 [batch][num_q_heads][128]; may not alias q. */
+WUSHKV_API int wushkv_transform_query(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                           int32_t num_kv_heads, const float* Tk_invT, float* q_out, void* stream);
+
+/* Bytes of decode workspace needed for wushkv_decode_attention with the same
+ * cache shape, num_q_heads and num_splits (0 = the automatic split count).
+ * Returns 0 for invalid arguments.  Host only; no CUDA call. */
+WUSHKV_API size_t wushkv_decode_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads,
+                                     int32_t num_splits);
+
+/* Split-K GQA decode attention directly over the packed cache ([ai4s 5]: serving
+ * with grouped-query attention over a 2-bit cache; long contexts [ai4s 4]).
+ * For each sequence b and query head h (KV head h / g):
+ *   s_t = softmax_scale * q_t[b][h] . k_hat_t,  t < ctx_len[b]
+ *   out[b][h] = sum_t softmax(s)_t * v_hat_t   (in the transformed value basis).
+ *   q_t        : fp32 [batch][num_q_heads][128] from wushkv_transform_query.
+ *   ctx_len    : int32 [batch] (device), cached tokens per sequence; 0 gives a zero
+ *                row; values > capacity are clamped (WUSHKV_STATUS_CTX_OVERFLOW).
+ *   out        : fp32 [batch][num_q_heads][128].
+ *   workspace  : scratch of at least wushkv_decode_workspace_bytes() bytes,
+ *                16-byte aligned; contents on entry are ignored.
+ *   num_splits : splits of each sequence's context (0 = automatic). */
+WUSHKV_API int wushkv_decode_attention(const wushkv_cache* cache, const float* q_t, int32_t num_q_heads,
+                            const int32_t* ctx_len, float softmax_scale, float* out,
+                            void* workspace, size_t workspace_bytes, int32_t num_splits,
+                            int32_t* status, void* stream);
+
+/* Static text for a wushkv_error code, or the last CUDA error text for WUSHKV_ERR_CUDA
+ * on the calling thread. */
+WUSHKV_API const char* wushkv_strerror(int code);
+
+/* Library version string. */
+WUSHKV_API const char* wushkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WUSHKV_H_ */

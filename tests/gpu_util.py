@@ -1,0 +1,59 @@
+"""Helpers shared by the GPU parity tests: moving caches between the oracle's numpy
+layout and the library's tensors, and the comparison rules the parity bar states."""
+import numpy as np
+import torch
+
+import decode_attention_quant_b200 as dq
+import oracle.wushkv_oracle as orc
+
+
+def to_numpy64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float32).numpy().astype(np.float64)
+
+
+def cache_to_gpu(ocache, kind, bits, alpha=0.0, rank_lo=2, rank_hi=125) -> dq.PackedCache:
+    b, h, t, _ = ocache["k_codes"].shape
+    tens = {k: torch.from_numpy(np.ascontiguousarray(v.view(np.int16) if v.dtype == np.uint16 else v)).cuda()
+            for k, v in ocache.items()}
+    return dq.PackedCache(b, h, t, kind, bits, alpha, rank_lo, rank_hi, tensors=tens)
+
+
+def cache_to_numpy(cache: dq.PackedCache):
+    return {"k_codes": cache.k_codes.cpu().numpy(), "v_codes": cache.v_codes.cpu().numpy(),
+            "k_meta": cache.k_meta.cpu().numpy().view(np.uint16),
+            "v_meta": cache.v_meta.cpu().numpy().view(np.uint16)}
+
+
+def fp16_midpoint_distance(pre):
+    """|pre - nearest midpoint between two adjacent fp16 values| (float64)."""
+    pre = np.asarray(pre, np.float64)
+    r = orc.fp16_round(pre)
+    h = np.abs(r).astype(np.float16)
+    up = np.nextafter(h, np.float16(np.inf)).astype(np.float64)
+    dn = np.nextafter(h, np.float16(0)).astype(np.float64)
+    a = np.abs(r)
+    return np.minimum(np.abs(np.abs(pre) - (a + up) / 2), np.abs(np.abs(pre) - (a + dn) / 2))
+
+
+def quest_boundary_distance(x, delta, bits):
+    """Distance of each x to the nearest decision threshold j*Delta."""
+    half = 1 << (bits - 1)
+    d = np.asarray(delta, np.float64)[..., None]
+    j = np.clip(np.round(x / np.where(d == 0, 1, d)), -(half - 1), half - 1)
+    return np.abs(x - j * d)
+
+
+def affine_boundary_distance(x, scale, zero, bits):
+    levels = (1 << bits) - 1
+    s = np.asarray(scale, np.float64)[..., None]
+    z = np.asarray(zero, np.float64)[..., None]
+    j = np.clip(np.floor((x - z) / np.where(s == 0, 1, s)), 0, levels - 1)
+    return np.abs(x - (z + (j + 0.5) * s))
+
+
+def attention_errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    max_abs = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+    return max_abs, rel_l2

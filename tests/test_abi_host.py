@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the header
+declares, and rejects bad arguments before anything reaches a GPU.  None of these
+calls launches a kernel, so they run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_attention_quant_b200 as dq
+from decode_attention_quant_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "wushkv.h")
+
+
+def _declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wushkv_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    lib = dq.library()
+    declared = _declared_symbols()
+    assert declared == sorted(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_strerror():
+    lib = dq.library()
+    assert lib.wushkv_version().startswith(b"wushkv")
+    for code in (0, -1, -2, -3, -4, -5, 7):
+        assert isinstance(_lib.strerror(code), str)
+
+
+def _desc(**kw):
+    qp = _lib.QuantParams(kw.pop("kind", 0), kw.pop("bits", 2), kw.pop("alpha", 1.99), kw.pop("rlo", 2),
+                          kw.pop("rhi", 125))
+    fields = dict(k_codes=0x10000, v_codes=0x20000, k_meta=0x30000, v_meta=0x40000, batch=2,
+                  num_kv_heads=2, capacity=256, head_dim=128)
+    fields.update(kw)
+    return _lib.CacheDesc(fields["k_codes"], fields["v_codes"], fields["k_meta"], fields["v_meta"],
+                          fields["batch"], fields["num_kv_heads"], fields["capacity"], fields["head_dim"], qp)
+
+
+BAD_CACHES = [
+    (dict(head_dim=64), _lib.ERR_UNSUPPORTED),
+    (dict(bits=1), _lib.ERR_UNSUPPORTED),
+    (dict(bits=5), _lib.ERR_UNSUPPORTED),
+    (dict(kind=7), _lib.ERR_UNSUPPORTED),
+    (dict(batch=0), _lib.ERR_INVALID),
+    (dict(capacity=0), _lib.ERR_INVALID),
+    (dict(alpha=0.0), _lib.ERR_INVALID),
+    (dict(alpha=float("nan")), _lib.ERR_INVALID),
+    (dict(kind=1, rlo=5, rhi=4), _lib.ERR_INVALID),
+    (dict(kind=1, rlo=10, rhi=120), _lib.ERR_UNSUPPORTED),
+    (dict(k_codes=0), _lib.ERR_INVALID),
+    (dict(v_codes=0x20008), _lib.ERR_MISALIGNED),
+    (dict(k_meta=0x30002), _lib.ERR_MISALIGNED),
+]
+
+
+@pytest.mark.parametrize("kw,code", BAD_CACHES)
+def test_append_rejects_bad_cache(kw, code):
+    lib = dq.library()
+    d = _desc(**kw)
+    rc = lib.wushkv_quantize_append(ctypes.byref(d), 0x50000, 0x60000, 0, 4, 0x70000, None, None, None)
+    assert rc == code
+    assert lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 0) == 0
+
+
+def test_append_rejects_bad_arguments():
+    lib = dq.library()
+    d = _desc()
+    call = lib.wushkv_quantize_append
+    assert call(None, 0x50000, 0x60000, 0, 4, 0x70000, None, None, None) == _lib.ERR_INVALID
+    assert call(ctypes.byref(d), 0x50000, 0x60000, 9, 4, 0x70000, None, None, None) == _lib.ERR_UNSUPPORTED
+    assert call(ctypes.byref(d), 0x50000, 0x60000, 0, 0, 0x70000, None, None, None) == _lib.ERR_INVALID
+    assert call(ctypes.byref(d), None, 0x60000, 0, 4, 0x70000, None, None, None) == _lib.ERR_INVALID
+    assert call(ctypes.byref(d), 0x50000, 0x60000, 0, 4, None, None, None, None) == _lib.ERR_INVALID
+    assert call(ctypes.byref(d), 0x50004, 0x60000, 0, 4, 0x70000, None, None, None) == _lib.ERR_MISALIGNED
+    assert call(ctypes.byref(d), 0x50000, 0x60000, 0, 4, 0x70002, None, None, None) == _lib.ERR_MISALIGNED
+    assert call(ctypes.byref(d), 0x50000, 0x60000, 0, 4, 0x70000, 0x80004, None, None) == _lib.ERR_MISALIGNED
+
+
+def test_transform_query_rejects_bad_arguments():
+    f = dq.library().wushkv_transform_query
+    assert f(0x1000, 3, 2, 32, 8, 0x2000, 0x3000, None) == _lib.ERR_UNSUPPORTED
+    assert f(0x1000, 0, 2, 30, 8, 0x2000, 0x3000, None) == _lib.ERR_INVALID
+    assert f(0x1000, 0, 2, 96, 4, 0x2000, 0x3000, None) == _lib.ERR_UNSUPPORTED   # g = 24
+    assert f(0x1000, 0, 0, 32, 8, 0x2000, 0x3000, None) == _lib.ERR_INVALID
+    assert f(0x1000, 0, 2, 32, 8, None, 0x3000, None) == _lib.ERR_INVALID
+    assert f(0x1000, 0, 2, 32, 8, 0x2000, 0x1000, None) == _lib.ERR_INVALID       # aliasing
+    assert f(0x1004, 0, 2, 32, 8, 0x2000, 0x3000, None) == _lib.ERR_MISALIGNED
+
+
+def test_decode_rejects_bad_arguments():
+    lib = dq.library()
+    d = _desc()
+    need = lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 0)
+    assert need > 0
+    assert lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 3) == 2 * 4 * 3 * 132 * 4
+    assert lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 3, 0) == 0
+    f = lib.wushkv_decode_attention
+    ok = (ctypes.byref(d), 0x1000, 4, 0x2000, 0.1, 0x3000, 0x4000, need, 0, None, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["c", "q", "hq", "ctx", "scale", "out", "ws", "wsb", "ns", "st", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+
+    assert call(ws=0x4000, wsb=need - 1) == _lib.ERR_WORKSPACE
+    assert call(q=None) == _lib.ERR_INVALID
+    assert call(hq=5) == _lib.ERR_INVALID
+    assert call(hq=6) == _lib.ERR_UNSUPPORTED
+    assert call(ns=-1) == _lib.ERR_INVALID
+    assert call(scale=float("inf")) == _lib.ERR_INVALID
+    assert call(out=0x3004) == _lib.ERR_MISALIGNED
+    assert call(ctx=0x2002) == _lib.ERR_MISALIGNED
+    assert call(st=0x5002) == _lib.ERR_MISALIGNED
