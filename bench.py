@@ -93,7 +93,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.rows.append([s.strip() for s in line.split(",")])
+            self.rows.append((time.time(), [s.strip() for s in line.split(",")]))
+
+    def mark(self):
+        return time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -103,16 +106,17 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in self.rows if len(r) > 8 and r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in self.rows if len(r) > 8 and r[2].replace(".", "").isdigit()]
+    def summary(self, t_from=0.0, t_to=float("inf"), window=""):
+        rows = [r for t, r in self.rows if t_from <= t <= t_to and len(r) > 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "window": window}
+        num = lambda v: v.replace(".", "").isdigit()  # noqa: E731
+        sm = [float(r[1]) for r in rows if num(r[1])]
+        mx = [float(r[2]) for r in rows if num(r[2])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows if len(r) > 8 for i in range(4)
-                          if r[5 + i].lower() in ("active", "1")})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() in ("active", "1")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(rows), "window": window}
 
 
 # ------------------------------------------------------------------- distributed
@@ -195,14 +199,21 @@ def run_ours(args, rank, world, local):
         dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
 
     launches_per_step = 2 + 1 + 2
+    clk = ClockSampler(local).__enter__()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    # untimed soak so that the clock sampler (100 ms period) sees the GPU under this load
+    soak_from = time.time()
+    while time.time() - soak_from < 1.0:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize()
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    if True:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
@@ -216,6 +227,8 @@ def run_ours(args, rank, world, local):
             ev[i][3].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
+    timed_to = time.time()
+    clk.__exit__(None, None, None)
     barrier(world)
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
@@ -276,7 +289,7 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clk.summary(soak_from, timed_to, "1 s untimed soak of the same step + the timed steps"),
         "device_status": st,
     }
     return res
@@ -327,7 +340,7 @@ def oracle_sample(w, pairs, seed=0):
     g = w.group
     k_new = gen.keys(w, 0, 1, w.ctx - 1, 1).float().numpy()[:, :, :1].repeat(pairs, axis=2).astype(np.float64)
     v_new = gen.values(w, 0, 1, w.ctx - 1, 1).float().numpy()[:, :, :1].repeat(pairs, axis=2).astype(np.float64)
-    q = gen.queries(w).float().numpy()[:1, :pairs * g].astype(np.float64)
+    q = np.tile(gen.queries(w).float().numpy()[:1, :g].astype(np.float64), (1, pairs, 1))
     return c, k_new, v_new, q, np.stack([tk[0]] * pairs), np.stack([tinv[0]] * pairs)
 
 
@@ -357,7 +370,7 @@ def oracle_threads():
         return 1
 
 
-def cpu_baseline(w, pairs=32):
+def cpu_baseline(w, pairs=64):
     dt, by = time_oracle(w, pairs)
     return {"value": round(by / dt / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(), "kind": "oracle",
             "sample": f"{pairs} of {w.batch * w.num_kv_heads} (sequence, KV head) pairs at ctx {w.ctx}: "

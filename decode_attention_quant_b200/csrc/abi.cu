@@ -8,6 +8,9 @@
 #include "wushkv_launch.h"
 
 namespace wushkv {
+cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
+                                      const int32_t* start_pos, const float* Tk, int32_t* status,
+                                      cudaStream_t stream);
 cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new, const void* v_new,
                                         int in_dtype, int n_new, const int32_t* start_pos,
                                         const float* Tk, int32_t* status, cudaStream_t stream);
@@ -24,8 +27,9 @@ int cuda_fail(cudaError_t e) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Shape, quantizer and pointer checks shared by every call that takes a cache.
-int check_cache(const wushkv_cache* c) {
+// Shape, quantizer and pointer checks shared by every call that takes a cache.  The
+// clip multiplier only matters when quantizing (append), not when reading the cache.
+int check_cache(const wushkv_cache* c, bool quantizing) {
   if (c == nullptr) return WUSHKV_ERR_INVALID;
   if (c->head_dim != WUSHKV_HEAD_DIM) return WUSHKV_ERR_UNSUPPORTED;
   if (c->qp.bits < 2 || c->qp.bits > 4) return WUSHKV_ERR_UNSUPPORTED;
@@ -33,7 +37,7 @@ int check_cache(const wushkv_cache* c) {
   if (c->batch <= 0 || c->num_kv_heads <= 0 || c->capacity <= 0) return WUSHKV_ERR_INVALID;
   if ((int64_t)c->batch * c->num_kv_heads * c->capacity > (int64_t)1 << 40) return WUSHKV_ERR_INVALID;
   if (c->qp.kind == WUSHKV_QUEST_INT) {
-    if (!(c->qp.clip_alpha > 0.0) || !std::isfinite(c->qp.clip_alpha)) return WUSHKV_ERR_INVALID;
+    if (quantizing && (!(c->qp.clip_alpha > 0.0) || !std::isfinite(c->qp.clip_alpha))) return WUSHKV_ERR_INVALID;
   } else {
     if (c->qp.rank_lo < 0 || c->qp.rank_hi > WUSHKV_HEAD_DIM - 1) return WUSHKV_ERR_INVALID;
     if (c->qp.rank_lo >= c->qp.rank_hi) return WUSHKV_ERR_INVALID;
@@ -60,7 +64,7 @@ extern "C" {
 int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const void* v_new,
                            int32_t in_dtype, int32_t n_new, const int32_t* start_pos,
                            const float* Tk, int32_t* status, void* stream) {
-  int rc = check_cache(cache);
+  int rc = check_cache(cache, true);
   if (rc != WUSHKV_OK) return rc;
   if (in_dtype != WUSHKV_BF16 && in_dtype != WUSHKV_FP32) return WUSHKV_ERR_UNSUPPORTED;
   if (n_new <= 0 || !k_new || !v_new || !start_pos) return WUSHKV_ERR_INVALID;
@@ -68,8 +72,14 @@ int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const v
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(start_pos, 4)) return WUSHKV_ERR_MISALIGNED;
   if (Tk != nullptr && !aligned(Tk, 16)) return WUSHKV_ERR_MISALIGNED;
   if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
-  cudaError_t e = wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos,
-                                                      Tk, status, static_cast<cudaStream_t>(stream));
+  // bf16 rows (the serving path) go through TMA + tcgen05; fp32 rows (exact pre-transformed
+  // values, used to test the quantizer alone) through the per-row kernel.  Both share the
+  // quantizer code.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = in_dtype == WUSHKV_BF16
+                      ? wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st)
+                      : wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos, Tk,
+                                                            status, st);
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 
@@ -87,7 +97,7 @@ int wushkv_transform_query(const void* q, int32_t q_dtype, int32_t batch, int32_
 }
 
 size_t wushkv_decode_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads, int32_t num_splits) {
-  if (check_cache(cache) != WUSHKV_OK) return 0;
+  if (check_cache(cache, false) != WUSHKV_OK) return 0;
   if (check_heads(num_q_heads, cache->num_kv_heads) != WUSHKV_OK) return 0;
   if (num_splits < 0) return 0;
   return wushkv::decode_workspace_bytes(*cache, num_q_heads, num_splits);
@@ -97,7 +107,7 @@ int wushkv_decode_attention(const wushkv_cache* cache, const float* q_t, int32_t
                             const int32_t* ctx_len, float softmax_scale, float* out,
                             void* workspace, size_t workspace_bytes, int32_t num_splits,
                             int32_t* status, void* stream) {
-  int rc = check_cache(cache);
+  int rc = check_cache(cache, false);
   if (rc != WUSHKV_OK) return rc;
   rc = check_heads(num_q_heads, cache->num_kv_heads);
   if (rc != WUSHKV_OK) return rc;

@@ -98,17 +98,15 @@ __global__ void __launch_bounds__(kRows) append_rows_kernel(RowArgs a) {
 
   const int f = tile * kRows + tid;
   if (f >= a.total_rows) return;
-  float x[kHeadDim];
-#pragma unroll
-  for (int j = 0; j < kHeadDim; ++j) x[j] = xs[tid * kPad + j];
+  SmemRowLoader ld{xs + tid * kPad};
 
   uint32_t w[4 * BITS];
   uint16_t m0 = 0, m1 = 0;
   int32_t flags = 0;
   if (KIND == WUSHKV_QUEST_INT) {
-    quest_quantize<BITS>(x, a.alpha, w, m0, flags);
+    quest_quantize<BITS>(ld, a.alpha, w, m0, flags);
   } else {
-    affine_quantize<BITS, 3>(x, a.rank_lo, a.rank_hi, w, m0, m1, flags);
+    affine_quantize<BITS, 3>(ld, a.rank_lo, a.rank_hi, w, m0, m1, flags);
   }
 
   const int b = f / a.n_new, t = f - b * a.n_new;

@@ -35,6 +35,22 @@ __device__ __forceinline__ void put_code(uint32_t (&w)[4 * BITS], int i, uint32_
   if (sh + BITS > 32) w[wi + 1] |= c >> (32 - sh);
 }
 
+// Same as put_code for an index only known at run time (selects over the words so the
+// array stays in registers).
+template <int BITS>
+__device__ __forceinline__ void put_code_dyn(uint32_t (&w)[4 * BITS], int i, uint32_t c) {
+  const int o = BITS * i;
+  const int wi = o >> 5;
+  const int sh = o & 31;
+  const uint32_t lo = c << sh;
+  const uint32_t hi = (sh + BITS > 32) ? (c >> (32 - sh)) : 0u;
+#pragma unroll
+  for (int q = 0; q < 4 * BITS; ++q) {
+    if (q == wi) w[q] |= lo;
+    if (q == wi + 1) w[q] |= hi;
+  }
+}
+
 template <int BITS>
 __device__ __forceinline__ void clear_words(uint32_t (&w)[4 * BITS]) {
 #pragma unroll
@@ -48,84 +64,101 @@ __device__ __forceinline__ double quest_pre(double sumsq, double alpha, int bits
   return alpha * rms * ldexp(1.0, 1 - bits);
 }
 
+// The quantizers read a group as four chunks of 32 values through a loader
+// `ld(c, v)` (c = 0..3, v = float[32]): once for the statistics, once for the codes,
+// and again only in the rare exact fallbacks.  Re-reading from shared or tensor
+// memory keeps the register footprint at one chunk.  Loaders may be warp-collective
+// (tensor-memory loads), so every lane of the calling warp runs the same loads: there
+// is no early exit, degenerate groups are handled arithmetically, and the fallbacks
+// run for the whole warp when any lane needs them (exact results are always valid).
+constexpr int kChunk = 32;
+
 // ---------------------------------------------------------------------------- QuEST
-template <int BITS>
-__device__ __forceinline__ void quest_quantize(const float (&x)[kHeadDim], double alpha,
-                                               uint32_t (&w)[4 * BITS], uint16_t& delta_bits,
-                                               int32_t& flags) {
+template <int BITS, class Loader>
+__device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint32_t (&w)[4 * BITS],
+                                               uint16_t& delta_bits, int32_t& flags) {
   constexpr int kHalf = 1 << (BITS - 1);
   constexpr int kMaxCode = (1 << BITS) - 1;
+  const unsigned mask = __activemask();
   float s[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) s[k] = 0.f;
 #pragma unroll
-  for (int i = 0; i < kHeadDim; ++i) s[i & 7] = fmaf(x[i], x[i], s[i & 7]);
+  for (int c = 0; c < 4; ++c) {
+    float v[kChunk];
+    ld(c, v);
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) s[i & 7] = fmaf(v[i], v[i], s[i & 7]);
+  }
   const double sum_fast = (((double)s[0] + (double)s[1]) + ((double)s[2] + (double)s[3])) +
                           (((double)s[4] + (double)s[5]) + ((double)s[6] + (double)s[7]));
   if (!isfinite(sum_fast)) flags |= WUSHKV_STATUS_NONFINITE;
   const double pre_fast = quest_pre(sum_fast, alpha, BITS);
   uint16_t h = f64_to_f16_bits(pre_fast * (1.0 - kStepMargin));
-  if (h != f64_to_f16_bits(pre_fast * (1.0 + kStepMargin))) {
+  const bool ambiguous = h != f64_to_f16_bits(pre_fast * (1.0 + kStepMargin));
+  if (__any_sync(mask, ambiguous)) {  // fp64 sum of the exact squares
     double sum = 0.0;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[kChunk];
+      ld(c, v);
 #pragma unroll
-    for (int i = 0; i < kHeadDim; ++i) sum = fma((double)x[i], (double)x[i], sum);
+      for (int i = 0; i < kChunk; ++i) sum = fma((double)v[i], (double)v[i], sum);
+    }
     h = f64_to_f16_bits(quest_pre(sum, alpha, BITS));
   }
   delta_bits = h;
   const float delta = f16_bits_to_f32(h);
   if (isinf(delta)) flags |= WUSHKV_STATUS_META_OVERFLOW;
-  clear_words<BITS>(w);
-  if (delta == 0.f) {
-#pragma unroll
-    for (int i = 0; i < kHeadDim; ++i) put_code<BITS>(w, i, kHalf);
-    return;
-  }
-  const float inv = __frcp_rn(delta);
+  // Delta == 0 (or overflowed): a zero reciprocal puts every value at code 2^(b-1)
+  const float inv = (delta == 0.f || isinf(delta)) ? 0.f : __frcp_rn(delta);
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
   const float m = kMagic + (float)kHalf;
   uint32_t mism = 0u;
+  clear_words<BITS>(w);
 #pragma unroll
-  for (int i = 0; i < kHeadDim; ++i) {
-    const float y1 = __fmaf_rd(x[i], inv_dn, m);
-    const float y2 = __fmaf_rd(x[i], inv_up, m);
-    mism |= f2u(y1) ^ f2u(y2);
-    const int32_t c = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-    put_code<BITS>(w, i, (uint32_t)c);
+  for (int c = 0; c < 4; ++c) {
+    float v[kChunk];
+    ld(c, v);
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) {
+      const float y1 = __fmaf_rd(v[i], inv_dn, m);
+      const float y2 = __fmaf_rd(v[i], inv_up, m);
+      mism |= f2u(y1) ^ f2u(y2);
+      const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
+      put_code<BITS>(w, c * kChunk + i, (uint32_t)code);
+    }
   }
-  if (mism != 0u) {  // exact: count the thresholds j*Delta (exact in fp32) that x reaches
+  if (__any_sync(mask, mism != 0u)) {  // exact: count the thresholds j*Delta (exact in fp32)
     clear_words<BITS>(w);
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[kChunk];
+      ld(c, v);
 #pragma unroll
-    for (int i = 0; i < kHeadDim; ++i) {
-      uint32_t c = 0;
+      for (int i = 0; i < kChunk; ++i) {
+        uint32_t code = 0;
 #pragma unroll
-      for (int j = -(kHalf - 1); j < kHalf; ++j) c += (x[i] >= (float)j * delta) ? 1u : 0u;
-      put_code<BITS>(w, i, c);
+        for (int j = -(kHalf - 1); j < kHalf; ++j) code += (v[i] >= (float)j * delta) ? 1u : 0u;
+        if (inv == 0.f) code = kHalf;
+        put_code_dyn<BITS>(w, c * kChunk + i, code);
+      }
     }
   }
 }
 
 // ------------------------------------------------------------------ percentile affine
-// Smallest KSEL and largest KSEL values of the group, ascending / descending.
+// The KSEL smallest (ascending) and KSEL largest (descending) values seen so far.
 template <int KSEL>
-__device__ __forceinline__ void select_extremes(const float (&x)[kHeadDim], float (&lo)[KSEL],
-                                                float (&hi)[KSEL]) {
+__device__ __forceinline__ void select_update(float v, float (&lo)[KSEL], float (&hi)[KSEL]) {
 #pragma unroll
-  for (int k = 0; k < KSEL; ++k) {
-    lo[k] = __int_as_float(0x7f800000);
-    hi[k] = __int_as_float(0xff800000);
+  for (int k = KSEL - 1; k >= 1; --k) {
+    lo[k] = fminf(lo[k], fmaxf(lo[k - 1], v));
+    hi[k] = fmaxf(hi[k], fminf(hi[k - 1], v));
   }
-#pragma unroll
-  for (int i = 0; i < kHeadDim; ++i) {
-    const float v = x[i];
-#pragma unroll
-    for (int k = KSEL - 1; k >= 1; --k) {
-      lo[k] = fminf(lo[k], fmaxf(lo[k - 1], v));
-      hi[k] = fmaxf(hi[k], fminf(hi[k - 1], v));
-    }
-    lo[0] = fminf(lo[0], v);
-    hi[0] = fmaxf(hi[0], v);
-  }
+  lo[0] = fminf(lo[0], v);
+  hi[0] = fmaxf(hi[0], v);
 }
 
 template <int KSEL>
@@ -136,17 +169,28 @@ __device__ __forceinline__ float pick(const float (&a)[KSEL], int idx) {
   return r;
 }
 
-template <int BITS, int KSEL>
-__device__ __forceinline__ void affine_quantize(const float (&x)[kHeadDim], int rank_lo,
-                                                int rank_hi, uint32_t (&w)[4 * BITS],
-                                                uint16_t& scale_bits, uint16_t& zero_bits,
-                                                int32_t& flags) {
+template <int BITS, int KSEL, class Loader>
+__device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int rank_hi, uint32_t (&w)[4 * BITS],
+                                                uint16_t& scale_bits, uint16_t& zero_bits, int32_t& flags) {
   constexpr int kMaxCode = (1 << BITS) - 1;
+  const unsigned mask = __activemask();
   float lo_k[KSEL], hi_k[KSEL];
-  select_extremes<KSEL>(x, lo_k, hi_k);
+#pragma unroll
+  for (int k = 0; k < KSEL; ++k) {
+    lo_k[k] = __int_as_float(0x7f800000);
+    hi_k[k] = __int_as_float(0xff800000);
+  }
   float fsum = 0.f;
 #pragma unroll
-  for (int i = 0; i < kHeadDim; ++i) fsum += x[i];
+  for (int c = 0; c < 4; ++c) {
+    float v[kChunk];
+    ld(c, v);
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) {
+      select_update<KSEL>(v[i], lo_k, hi_k);
+      fsum += v[i];
+    }
+  }
   if (!isfinite(fsum)) flags |= WUSHKV_STATUS_NONFINITE;
   const float lo = pick<KSEL>(lo_k, rank_lo);
   const float hi = pick<KSEL>(hi_k, kHeadDim - 1 - rank_hi);
@@ -156,36 +200,56 @@ __device__ __forceinline__ void affine_quantize(const float (&x)[kHeadDim], int 
   const float sc = f16_bits_to_f32(scale_bits);
   const float z = f16_bits_to_f32(zero_bits);
   if (isinf(sc) || isinf(z)) flags |= WUSHKV_STATUS_META_OVERFLOW;
-  clear_words<BITS>(w);
-  if (sc == 0.f) return;  // all codes 0: x_hat = zero
-  const float inv = __frcp_rn(sc);
+  // scale == 0: a zero reciprocal puts every value at code 0 (x_hat = zero)
+  const float inv = (sc == 0.f || isinf(sc)) ? 0.f : __frcp_rn(sc);
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
   uint32_t mism = 0u;
+  clear_words<BITS>(w);
 #pragma unroll
-  for (int i = 0; i < kHeadDim; ++i) {
-    const float d = __fsub_rn(x[i], z);
-    const float y1 = __fmaf_rn(d, inv_dn, kMagic);
-    const float y2 = __fmaf_rn(d, inv_up, kMagic);
-    mism |= f2u(y1) ^ f2u(y2);
-    const int32_t c = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-    put_code<BITS>(w, i, (uint32_t)c);
+  for (int c = 0; c < 4; ++c) {
+    float v[kChunk];
+    ld(c, v);
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) {
+      const float d = __fsub_rn(v[i], z);
+      const float y1 = __fmaf_rn(d, inv_dn, kMagic);
+      const float y2 = __fmaf_rn(d, inv_up, kMagic);
+      mism |= f2u(y1) ^ f2u(y2);
+      const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
+      put_code<BITS>(w, c * kChunk + i, (uint32_t)code);
+    }
   }
-  if (mism != 0u) {  // exact: thresholds zero + (j + 1/2) scale are exact in fp64
+  if (__any_sync(mask, mism != 0u)) {  // exact: thresholds zero + (j + 1/2) scale are exact in fp64
     clear_words<BITS>(w);
     const double zd = (double)z, sd = (double)sc;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[kChunk];
+      ld(c, v);
 #pragma unroll
-    for (int i = 0; i < kHeadDim; ++i) {
-      const double xd = (double)x[i];
-      uint32_t c = 0;
+      for (int i = 0; i < kChunk; ++i) {
+        const double xd = (double)v[i];
+        uint32_t code = 0;
 #pragma unroll
-      for (int j = 0; j < kMaxCode; ++j) {
-        const double t = zd + ((double)j + 0.5) * sd;
-        c += (xd > t || (xd == t && (j & 1))) ? 1u : 0u;
+        for (int j = 0; j < kMaxCode; ++j) {
+          const double t = zd + ((double)j + 0.5) * sd;
+          code += (xd > t || (xd == t && (j & 1))) ? 1u : 0u;
+        }
+        if (inv == 0.f) code = 0;
+        put_code_dyn<BITS>(w, c * kChunk + i, code);
       }
-      put_code<BITS>(w, i, c);
     }
   }
 }
+
+// Loader over a group held in a shared-memory row of fp32 values.
+struct SmemRowLoader {
+  const float* row;
+  __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) v[i] = row[c * kChunk + i];
+  }
+};
 
 }  // namespace wushkv
