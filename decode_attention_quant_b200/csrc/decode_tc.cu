@@ -1,0 +1,638 @@
+// Split-K GQA decode attention directly over the packed cache, on the tensor cores.
+//
+// WUSH-KV serves grouped-query attention over a 2-bit cache (ai4snews summary,
+// paragraph 5) at long context (paragraph 4).  The codes are small integers, so
+// both contractions run exactly as integer MMAs (tcgen05.mma kind::i8, int32
+// accumulate) and the fp16 meta is applied afterwards:
+//   scores  s_t = tau * (scale_t * sum_c q'_c code_tc + zero_t * sum_c q'_c)
+//           sum_c q'_c code_tc = (M / (2^22 - 1)) * sum_c qi_c code_tc, with q' rounded
+//           to 23-bit integers qi = l0 + 2^8 l1 + 2^16 l2 split into three int8 limbs;
+//   values  o_c = sum_t p_t (zero_t + scale_t code_tc)
+//               = (F / 65535) * sum_t pi_t code_tc + sum_t p_t zero_t,
+//           with p_t scale_t rounded to 16-bit integers pi = u0 + 2^8 u1 (per tile and
+//           head, F = the tile's largest p_t scale_t) split into two uint8 limbs.
+// (QuEST: scale = Delta, zero = -(2^(b-1) - 1/2) Delta.)  The softmax is online in the
+// log2 domain across 128-token tiles.
+//
+// One CTA = one (sequence, KV head, split).  Warp roles:
+//   warp 0      bulk copies of the tile's packed K and V codes into a 4-stage ring
+//   warp 1      TMEM allocation, MMA issue (one thread)
+//   warps 2-5   token warps (thread = token of the tile): unpack K codes to u8 in
+//               tensor memory (A of the score MMA) and V codes to u8 in shared memory
+//               (A of the value MMA, channel-major), then scores, online softmax and
+//               the probability limbs (B of the value MMA)
+//   warps 6-9   channel warps (thread = channel): rescale and accumulate the value
+//               MMA's int32 result into fp32 outputs
+// 2- and 4-bit codes are widened to bytes with two logic ops per 4 codes, which
+// permutes channels inside each 16 (8) channel block; the query limbs and the output
+// channels use the same permutation, so the contraction is unchanged.
+#include <math_constants.h>
+
+#include <cmath>
+
+#include "sm100.cuh"
+#include "tmap.h"
+#include "wushkv_common.cuh"
+#include "wushkv_launch.h"
+
+namespace wushkv {
+namespace {
+
+using namespace sm100;
+
+constexpr int kTile = 128;
+constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kPartialStride = 132;   // m (log2 domain), l, pad, pad, o[128]
+constexpr int kRing = 4;              // per-tile (corr, F) slots shared with the channel warps
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kQScale = 4194303.0f; // 2^22 - 1
+
+__host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
+__host__ __device__ constexpr int pow2cols(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
+
+template <int BITS, int G>
+struct Cfg {
+  static constexpr int kCode = 16 * BITS;                  // packed bytes per token row
+  static constexpr int kStage = 2 * kTile * kCode;         // K and V codes of one tile
+  static constexpr int NK = round16(3 * G);                // score MMA N (3 limbs per head)
+  static constexpr int NV = round16(2 * G);                // value MMA N (2 limbs per head)
+  static constexpr int kColAk = 0;                         // 2 x 32 columns (u8 x 128 channels)
+  static constexpr int kColS = 64;                         // 2 x NK
+  static constexpr int kColO = 64 + 2 * NK;                // 2 x NV
+  static constexpr int kCols = pow2cols(64 + 2 * NK + 2 * NV);
+  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr int kOffStage = 0;
+  static constexpr int kOffAv = (kOffStage + kStages * kStage + 1023) / 1024 * 1024;   // 2 x 16 KB
+  static constexpr int kOffBv = kOffAv + 2 * kTile * 128;                              // 2 x NV rows
+  static constexpr int kOffBk = kOffBv + 2 * NV * 128;                                 // NK rows
+  static constexpr int kOffMisc = kOffBk + NK * 128;
+  static constexpr int kMiscBytes = 4096;
+  static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
+};
+
+struct DecArgs {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const uint16_t* k_meta;
+  const uint16_t* v_meta;
+  int hkv, hq, capacity, num_splits;
+  const float* q;          // [B][Hq][128]
+  const int32_t* ctx_len;
+  float scale_log2;        // softmax scale * log2(e)
+  float* ws;               // [B][Hq][S][132]
+  int32_t* status;
+};
+
+struct Misc {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t unp_full[2], unp_empty[2], s_full[2], s_empty[2], bv_full[2], o_full[2], o_empty[2];
+  uint64_t red_bar[2], fin_bar, fin_done;
+  uint32_t tmem_base;
+  int abort;
+  float red[2][4][33];        // per tile parity, per token warp: max s and max (s + log2 scale) per head
+  float qscale[16], qsum[16];
+  float ring_corr[kRing][16], ring_f[kRing][16];
+  float fin_l[16], fin_z[16], fin_m[16];
+  float fin_part[4][2][16];   // per token warp: l and z partial sums
+};
+
+// position p of a widened code row <-> channel
+template <int BITS>
+__device__ __forceinline__ int channel_of(int p) {
+  if (BITS == 2) return (p & ~15) | ((p & 3) << 2) | ((p >> 2) & 3);
+  if (BITS == 4) return (p & ~7) | ((p & 3) << 1) | ((p >> 2) & 1);
+  return p;
+}
+
+// Packed row (16*BITS bytes at `row`) -> 32 words of four u8 codes (K order as above).
+template <int BITS>
+__device__ __forceinline__ void widen_row(const uint8_t* row, int r, uint32_t (&u)[32]) {
+  constexpr int kWords = 4 * BITS;
+  uint32_t w[kWords];
+#pragma unroll
+  for (int q = 0; q < BITS; ++q) {              // 16-byte pieces, rotated by row to spread banks
+    const int piece = (q + r) % BITS;
+    const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * piece);
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) {
+      if (k == piece) { w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w; }
+    }
+  }
+  if (BITS == 2) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[4 * j + k] = (w[j] >> (2 * k)) & 0x03030303u;
+  } else if (BITS == 4) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) u[2 * j + k] = (w[j] >> (4 * k)) & 0x0F0F0F0Fu;
+  } else {
+#pragma unroll
+    for (int g = 0; g < 32; ++g) {              // codes 4g..4g+3: 12 bits at bit 12g
+      const int bit = 12 * g, wi = bit >> 5, sh = bit & 31;
+      const uint32_t hi = (wi + 1 < kWords) ? w[wi + 1] : 0u;
+      const uint32_t f = __funnelshift_r(w[wi], hi, sh) & 0xFFFu;
+      const uint32_t a = (f & 0x3Fu) | ((f & 0xFC0u) << 10);
+      u[g] = (a & 0x00070007u) | ((a & 0x00380038u) << 5);
+    }
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void meta_pair(uint32_t raw, int bits, float& scale, float& zero) {
+  if (KIND == WUSHKV_QUEST_INT) {
+    scale = f16_bits_to_f32((uint16_t)raw);
+    zero = -((float)(1 << (bits - 1)) - 0.5f) * scale;
+  } else {
+    scale = f16_bits_to_f32((uint16_t)(raw & 0xffffu));
+    zero = f16_bits_to_f32((uint16_t)(raw >> 16));
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ uint32_t load_meta(const uint16_t* meta, size_t row) {
+  if (KIND == WUSHKV_QUEST_INT) return (uint32_t)__ldg(meta + row);
+  return __ldg(reinterpret_cast<const uint32_t*>(meta) + row);
+}
+
+// byte (row n, column k) of a K-major operand stored as 128-byte rows, 128B-swizzled
+__device__ __forceinline__ int kmajor_off(int n, int k) {
+  return (n >> 3) * 1024 + (n & 7) * 128 + ((((k >> 4) ^ (n & 7)) & 7) << 4) + (k & 15);
+}
+
+template <int BITS, int KIND, int G>
+__global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(DecArgs a) {
+  using C = Cfg<BITS, G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage = smem + C::kOffStage;
+  uint8_t* av = smem + C::kOffAv;
+  uint8_t* bv = smem + C::kOffBv;
+  uint8_t* bk = smem + C::kOffBk;
+  Misc* ms = reinterpret_cast<Misc*>(smem + C::kOffMisc);
+  volatile int* abort = &ms->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
+  int L = __ldg(a.ctx_len + b);
+  if (L > a.capacity) {
+    if (split == 0 && kv == 0 && threadIdx.x == 0) report(a.status, WUSHKV_STATUS_CTX_OVERFLOW);
+    L = a.capacity;
+  }
+  if (L < 0) L = 0;
+  const int tiles_all = (L + kTile - 1) / kTile;
+  const int per = (tiles_all + a.num_splits - 1) / a.num_splits;
+  const int tile0 = split * per;
+  const int n = max(0, min(per, tiles_all - tile0));
+  const size_t pair = (size_t)b * a.hkv + kv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ms->full[s], 1);
+      mbar_init(&ms->empty[s], 4);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&ms->unp_full[u], 4);
+      mbar_init(&ms->unp_empty[u], 1);
+      mbar_init(&ms->s_full[u], 1);
+      mbar_init(&ms->s_empty[u], 4);
+      mbar_init(&ms->bv_full[u], 4);
+      mbar_init(&ms->o_full[u], 1);
+      mbar_init(&ms->o_empty[u], 4);
+      mbar_init(&ms->red_bar[u], 4);
+    }
+    mbar_init(&ms->fin_bar, 4);
+    mbar_init(&ms->fin_done, 1);
+    ms->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ms->tmem_base, C::kCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2 && warp < 6) {
+    // query limbs (B of the score MMA): thread = code position p (channel channel_of(p))
+    const int p = threadIdx.x - 64;
+    const int c = channel_of<BITS>(p);
+    const int wq = p >> 5;
+    float qv[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      qv[h] = a.q[((size_t)b * a.hq + kv * G + h) * kHeadDim + c];
+      float mx = fabsf(qv[h]), sm = qv[h];
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        sm += __shfl_xor_sync(0xffffffffu, sm, off);
+      }
+      if (lane == 0) { ms->red[0][wq][h] = mx; ms->red[1][wq][h] = sm; }
+    }
+    named_barrier(1, 128);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mx = fmaxf(fmaxf(ms->red[0][0][h], ms->red[0][1][h]), fmaxf(ms->red[0][2][h], ms->red[0][3][h]));
+      const float inv = mx > 0.f ? kQScale / mx : 0.f;
+      const int qi = __float2int_rn(qv[h] * inv);           // |qi| <= 2^22 - 1
+      const int l0 = (int)(int8_t)(qi & 0xff);
+      const int r1 = (qi - l0) >> 8;
+      const int l1 = (int)(int8_t)(r1 & 0xff);
+      const int l2 = (r1 - l1) >> 8;                        // |l2| <= 64
+      bk[kmajor_off(h, p)] = (uint8_t)l0;
+      bk[kmajor_off(G + h, p)] = (uint8_t)l1;
+      bk[kmajor_off(2 * G + h, p)] = (uint8_t)l2;
+      if (p == 0) {
+        ms->qscale[h] = mx > 0.f ? mx / kQScale : 0.f;
+        ms->qsum[h] = (ms->red[1][0][h] + ms->red[1][1][h]) + (ms->red[1][2][h] + ms->red[1][3][h]);
+      }
+    }
+    for (int nrow = 3 * G; nrow < C::NK; ++nrow) bk[kmajor_off(nrow, p)] = 0;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- bulk loads
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!mbar_wait(&ms->empty[s], ph ^ 1, abort)) break;
+        const int t0 = (tile0 + i) * kTile;
+        const uint32_t bytes = (uint32_t)min(kTile, L - t0) * C::kCode;
+        mbar_arrive_expect_tx(&ms->full[s], 2 * bytes);
+        const size_t off = (pair * a.capacity + t0) * C::kCode;
+        bulk_load(stage + s * C::kStage, a.k_codes + off, bytes, &ms->full[s]);
+        bulk_load(stage + s * C::kStage + kTile * C::kCode, a.v_codes + off, bytes, &ms->full[s]);
+        ++issued;
+      }
+      volatile int no_abort = 0;
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_wait(&ms->full[i % kStages], (i / kStages) & 1, &no_abort);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
+      constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 0, 128, C::NV);
+      const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
+      auto value_mma = [&](int j) -> bool {
+        const int u = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&ms->bv_full[u], ph, abort)) return false;
+        if (!mbar_wait(&ms->o_empty[u], ph ^ 1, abort)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + ks * 4096, 16384, 1024, 2);
+          const uint64_t bdesc = desc_kmajor_sw128(bv_addr + u * C::NV * 128 + ks * 32);
+          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, ks > 0);
+        }
+        mma_commit(&ms->o_full[u]);
+        mma_commit(&ms->unp_empty[u]);
+        return true;
+      };
+      bool ok = true;
+      for (int i = 0; i < n && ok; ++i) {
+        const int u = i & 1;
+        const uint32_t ph = (i >> 1) & 1;
+        if (!mbar_wait(&ms->unp_full[u], ph, abort)) break;
+        if (!mbar_wait(&ms->s_empty[u], ph ^ 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_i8_ts(tmem + C::kColS + u * C::NK, tmem + C::kColAk + u * 32 + ks * 8,
+                    desc_kmajor_sw128(bk_addr + ks * 32), kIdK, ks > 0);
+        mma_commit(&ms->s_full[u]);
+        if (i >= 1) ok = value_mma(i - 1);
+      }
+      if (ok && n >= 1) value_mma(n - 1);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------- token warps
+    const int qd = warp & 3;                 // TMEM lane quarter
+    const int r = 32 * qd + lane;            // token row of the tile
+    float m_run[G], l_run[G], z_run[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; }
+    uint32_t kmeta_n = 0, vmeta_n = 0, kmeta_c = 0, vmeta_c = 0;
+
+    auto unpack = [&](int i) -> bool {
+      const int s = i % kStages;
+      const uint32_t sph = (i / kStages) & 1;
+      const int u = i & 1;
+      const uint32_t uph = (i >> 1) & 1;
+      const int t = (tile0 + i) * kTile + r;
+      if (t < L) {
+        kmeta_n = load_meta<KIND>(a.k_meta, pair * a.capacity + t);
+        vmeta_n = load_meta<KIND>(a.v_meta, pair * a.capacity + t);
+      }
+      if (!mbar_wait(&ms->full[s], sph, abort)) return false;
+      if (!mbar_wait(&ms->unp_empty[u], uph ^ 1, abort)) return false;
+      tc_fence_after();
+      uint32_t wv[32];
+      widen_row<BITS>(stage + s * C::kStage + r * C::kCode, r, wv);
+      tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + C::kColAk + u * 32, wv);
+      widen_row<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, r, wv);
+      uint8_t* arow = av + u * kTile * 128 + r * 128;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) =
+            make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
+      tmem_st_wait();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ms->unp_full[u]);
+        mbar_arrive(&ms->empty[s]);
+      }
+      return true;
+    };
+
+    auto softmax = [&](int i) -> bool {
+      const int u = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      const bool valid = (tile0 + i) * kTile + r < L;
+      if (!mbar_wait(&ms->s_full[u], ph, abort)) return false;
+      tc_fence_after();
+      uint32_t d[C::NK];
+      if constexpr (C::NK == 16) {
+        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + u * C::NK, *reinterpret_cast<uint32_t(*)[16]>(d));
+      } else {
+#pragma unroll
+        for (int c0 = 0; c0 < C::NK; c0 += 16)
+          tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + u * C::NK + c0,
+                    *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->s_empty[u]);
+      float ks, kz, vs, vz;
+      meta_pair<KIND>(kmeta_c, BITS, ks, kz);
+      meta_pair<KIND>(vmeta_c, BITS, vs, vz);
+      float s2[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int si = (int)d[h] + (int)d[G + h] * 256 + (int)d[2 * G + h] * 65536;
+        const float dot = fmaf(ks, (float)si * ms->qscale[h], kz * ms->qsum[h]);
+        s2[h] = valid ? dot * a.scale_log2 : -CUDART_INF_F;
+      }
+      // per head, across the 4 token warps: the tile's largest score and the largest
+      // log2 of (probability x value scale) before normalization
+      const int par = i & 1;
+      const float lvs = valid && vs > 0.f ? log2f(vs) : -CUDART_INF_F;
+#pragma unroll
+      for (int h = 0; h < 2 * G; ++h) {
+        float v = h < G ? s2[h] : s2[h - G] + lvs;
+#pragma unroll
+        for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        if (lane == 0) ms->red[par][qd][h] = v;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->red_bar[par]);
+      if (!mbar_wait(&ms->red_bar[par], (i >> 1) & 1, abort)) return false;
+      float corr[G], fpt[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mt = fmaxf(fmaxf(ms->red[par][0][h], ms->red[par][1][h]),
+                               fmaxf(ms->red[par][2][h], ms->red[par][3][h]));
+        const float mu = fmaxf(fmaxf(ms->red[par][0][G + h], ms->red[par][1][G + h]),
+                               fmaxf(ms->red[par][2][G + h], ms->red[par][3][G + h]));
+        const float mn = fmaxf(m_run[h], mt);
+        corr[h] = exp2f(m_run[h] - mn);       // 0 on the first tile
+        m_run[h] = mn;
+        // largest p * scale of the tile (slightly widened against log2/exp2 rounding)
+        fpt[h] = exp2f(mu - mn) * 1.000244140625f;
+      }
+      uint8_t* brow = bv + u * C::NV * 128;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float p = valid ? exp2f(s2[h] - m_run[h]) : 0.f;
+        l_run[h] = fmaf(l_run[h], corr[h], p);
+        z_run[h] = fmaf(z_run[h], corr[h], p * vz);
+        const float fq = fpt[h] > 0.f ? 65535.0f / fpt[h] : 0.f;
+        const int pi = min(__float2int_rn(p * vs * fq), 65535);
+        brow[kmajor_off(h, r)] = (uint8_t)(pi & 0xff);
+        brow[kmajor_off(G + h, r)] = (uint8_t)(pi >> 8);
+      }
+      if (threadIdx.x == 64) {
+        const int slot = i % kRing;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          ms->ring_corr[slot][h] = corr[h];
+          ms->ring_f[slot][h] = fpt[h] * (1.0f / 65535.0f);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->bv_full[u]);
+      return true;
+    };
+
+    // zero the padding rows of both value-limb buffers once
+    for (int nrow = 2 * G; nrow < C::NV; ++nrow) {
+      bv[kmajor_off(nrow, r)] = 0;
+      bv[C::NV * 128 + kmajor_off(nrow, r)] = 0;
+    }
+    fence_proxy_async_smem();
+    bool ok = n == 0 || unpack(0);
+    for (int i = 0; i < n && ok; ++i) {
+      kmeta_c = kmeta_n;
+      vmeta_c = vmeta_n;
+      if (i + 1 < n) ok = unpack(i + 1);
+      if (ok) ok = softmax(i);
+    }
+    // per-head totals of l and z over the 128 token threads
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float l = l_run[h], z = z_run[h];
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, off);
+        z += __shfl_xor_sync(0xffffffffu, z, off);
+      }
+      if (lane == 0) { ms->fin_part[qd][0][h] = l; ms->fin_part[qd][1][h] = z; }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ms->fin_bar);
+    if (threadIdx.x == 64) {
+      if (mbar_wait(&ms->fin_bar, 0, abort)) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          ms->fin_l[h] = (ms->fin_part[0][0][h] + ms->fin_part[1][0][h]) + (ms->fin_part[2][0][h] + ms->fin_part[3][0][h]);
+          ms->fin_z[h] = (ms->fin_part[0][1][h] + ms->fin_part[1][1][h]) + (ms->fin_part[2][1][h] + ms->fin_part[3][1][h]);
+          ms->fin_m[h] = m_run[h];
+        }
+      }
+      mbar_arrive(&ms->fin_done);
+    }
+  } else {
+    // ----------------------------------------------------------- channel warps
+    const int qd = warp & 3;
+    const int mpos = 32 * qd + lane;
+    float o[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) o[h] = 0.f;
+    for (int i = 0; i < n; ++i) {
+      const int u = i & 1;
+      const uint32_t ph = (i >> 1) & 1;
+      if (!mbar_wait(&ms->o_full[u], ph, abort)) break;
+      tc_fence_after();
+      uint32_t d[C::NV];
+#pragma unroll
+      for (int c0 = 0; c0 < C::NV; c0 += 16)
+        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColO + u * C::NV + c0,
+                  *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+      tmem_ld_wait();
+      const int slot = i % kRing;
+      float corr[G], fs[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        corr[h] = ms->ring_corr[slot][h];
+        fs[h] = ms->ring_f[slot][h];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->o_empty[u]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int di = (int)d[h] + ((int)d[G + h] << 8);
+        o[h] = fmaf(o[h], corr[h], fs[h] * (float)di);
+      }
+    }
+    mbar_wait(&ms->fin_done, 0, abort);
+    const int c = channel_of<BITS>(mpos);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float* dst = a.ws + (((size_t)b * a.hq + kv * G + h) * a.num_splits + split) * kPartialStride;
+      dst[4 + c] = o[h] + ms->fin_z[h];
+      if (mpos == 0) {
+        dst[0] = ms->fin_m[h];
+        dst[1] = ms->fin_l[h];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && ms->abort) report(a.status, WUSHKV_STATUS_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kCols);
+  }
+}
+
+// out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s   (log2-domain partials)
+__global__ void __launch_bounds__(kHeadDim) combine_log2_kernel(const float* __restrict__ ws, int num_splits,
+                                                               float* __restrict__ out) {
+  const size_t bh = blockIdx.x;
+  const int c = threadIdx.x;
+  const float* p = ws + bh * num_splits * kPartialStride;
+  float mx = -CUDART_INF_F;
+  for (int s = 0; s < num_splits; ++s) mx = fmaxf(mx, p[s * kPartialStride]);
+  float l = 0.f, o = 0.f;
+  if (mx > -CUDART_INF_F) {
+    for (int s = 0; s < num_splits; ++s) {
+      const float ms = p[s * kPartialStride];
+      if (ms == -CUDART_INF_F) continue;
+      const float w = exp2f(ms - mx);
+      l = fmaf(w, p[s * kPartialStride + 1], l);
+      o = fmaf(w, p[s * kPartialStride + 4 + c], o);
+    }
+  }
+  out[bh * kHeadDim + c] = l > 0.f ? o / l : 0.f;
+}
+
+template <int BITS, int KIND, int G>
+cudaError_t launch_g(const DecArgs& a, int batch, float* out, cudaStream_t stream) {
+  using C = Cfg<BITS, G>;
+  auto kern = decode_tc_kernel<BITS, KIND, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.num_splits, a.hkv, batch);
+  kern<<<grid, kThreads, C::kSmem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  combine_log2_kernel<<<batch * a.hq, kHeadDim, 0, stream>>>(a.ws, a.num_splits, out);
+  return cudaGetLastError();
+}
+
+template <int BITS, int KIND>
+cudaError_t launch_kind(const DecArgs& a, int batch, float* out, cudaStream_t stream) {
+  switch (a.hq / a.hkv) {
+    case 1: return launch_g<BITS, KIND, 1>(a, batch, out, stream);
+    case 2: return launch_g<BITS, KIND, 2>(a, batch, out, stream);
+    case 4: return launch_g<BITS, KIND, 4>(a, batch, out, stream);
+    case 8: return launch_g<BITS, KIND, 8>(a, batch, out, stream);
+    default: return launch_g<BITS, KIND, 16>(a, batch, out, stream);
+  }
+}
+
+template <int BITS>
+cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaStream_t stream) {
+  if (kind == WUSHKV_QUEST_INT) return launch_kind<BITS, WUSHKV_QUEST_INT>(a, batch, out, stream);
+  return launch_kind<BITS, WUSHKV_PCT_AFFINE>(a, batch, out, stream);
+}
+
+}  // namespace
+
+// Split count when the caller passes 0: the smallest count whose CTAs fill whole
+// waves of (SMs x 2 resident CTAs) to >= 95%, keeping >= 4 tiles per split; a small
+// problem gets one tile per CTA.
+int auto_num_splits(const wushkv_cache& c, int num_q_heads) {
+  (void)num_q_heads;
+  const int pairs = c.batch * c.num_kv_heads;
+  const int tiles = (c.capacity + kTile - 1) / kTile;
+  const int slots = 2 * num_sms(nullptr);
+  if ((long long)pairs * tiles <= slots) return tiles;
+  const int max_s = tiles >= 4 ? tiles / 4 : 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= max_s && s <= 256; ++s) {
+    const double w = (double)pairs * s / slots;
+    const double eff = w / std::ceil(w);
+    if (eff >= 0.95) return s;
+    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+  }
+  return best;
+}
+
+size_t decode_workspace_bytes(const wushkv_cache& c, int num_q_heads, int num_splits) {
+  const int s = num_splits > 0 ? num_splits : auto_num_splits(c, num_q_heads);
+  return (size_t)c.batch * num_q_heads * s * kPartialStride * sizeof(float);
+}
+
+cudaError_t launch_decode_attention(const wushkv_cache& c, const float* q_t, int num_q_heads,
+                                    const int32_t* ctx_len, float softmax_scale, float* out,
+                                    void* workspace, int num_splits, int32_t* status,
+                                    cudaStream_t stream) {
+  DecArgs a{};
+  a.k_codes = c.k_codes;
+  a.v_codes = c.v_codes;
+  a.k_meta = c.k_meta;
+  a.v_meta = c.v_meta;
+  a.hkv = c.num_kv_heads;
+  a.hq = num_q_heads;
+  a.capacity = c.capacity;
+  a.num_splits = num_splits > 0 ? num_splits : auto_num_splits(c, num_q_heads);
+  a.q = q_t;
+  a.ctx_len = ctx_len;
+  a.scale_log2 = softmax_scale * kLog2e;
+  a.ws = static_cast<float*>(workspace);
+  a.status = status;
+  switch (c.qp.bits) {
+    case 2: return launch_bits<2>(a, c.qp.kind, c.batch, out, stream);
+    case 3: return launch_bits<3>(a, c.qp.kind, c.batch, out, stream);
+    default: return launch_bits<4>(a, c.qp.kind, c.batch, out, stream);
+  }
+}
+
+}  // namespace wushkv

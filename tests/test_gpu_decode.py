@@ -81,15 +81,16 @@ def test_split_count_invariance_and_edges():
     q = torch.randn(bsz, hq, 128, generator=torch.Generator().manual_seed(3)).cuda()
     ctx = torch.tensor([1100, 0, 513], dtype=torch.int32, device="cuda")
     outs = [dq.decode_attention(cache, q, ctx, TAU, num_splits=s) for s in (1, 0, 3, 7, 9)]
+    # splits change only where the 16-bit probability limbs are rounded (per tile scale)
     for o in outs[1:]:
-        assert torch.allclose(o, outs[0], rtol=1e-5, atol=1e-6)
+        assert torch.allclose(o, outs[0], rtol=0, atol=5e-5), (o - outs[0]).abs().max()
     assert torch.all(outs[0][1] == 0)                 # ctx_len 0 -> zero rows
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     over = dq.decode_attention(cache, q, torch.tensor([5000, 0, 513], dtype=torch.int32, device="cuda"),
                                TAU, status=st)
     torch.cuda.synchronize()
     assert st.item() & dq.STATUS_CTX_OVERFLOW
-    assert torch.allclose(over, outs[0], rtol=1e-5, atol=1e-6)
+    assert torch.allclose(over, outs[0], rtol=0, atol=5e-5)
 
 
 @pytest.mark.parametrize("kind,bits,batch,hq,hkv,ctx", [
