@@ -129,10 +129,20 @@ __device__ __forceinline__ void quantize_store(Loader& ld, const TcArgs& a, int 
 // (exact: the remainders of a 24-bit significand split into 8 + 8 + 8 bits).
 __device__ __forceinline__ void split_transform(const float* __restrict__ tk, uint8_t* planes, int tid,
                                                 int nthreads) {
-  for (int q = tid; q < kHeadDim * kHeadDim / 4; q += nthreads) {
+  // all of this thread's loads first (independent, so their latencies overlap)
+  constexpr int kMaxPer = 16;
+  float4 t4[kMaxPer];
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int q = tid + k * nthreads;
+    if (q < kHeadDim * kHeadDim / 4) t4[k] = __ldg(reinterpret_cast<const float4*>(tk) + q);
+  }
+#pragma unroll
+  for (int k = 0; k < kMaxPer; ++k) {
+    const int q = tid + k * nthreads;
+    if (q >= kHeadDim * kHeadDim / 4) break;
     const int i = q >> 5, j = (q & 31) * 4;
-    const float4 t4 = __ldg(reinterpret_cast<const float4*>(tk) + q);
-    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+    const float tv[4] = {t4[k].x, t4[k].y, t4[k].z, t4[k].w};
     uint16_t p[3][4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

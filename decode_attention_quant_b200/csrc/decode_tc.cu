@@ -14,15 +14,18 @@
 // (QuEST: scale = Delta, zero = -(2^(b-1) - 1/2) Delta.)  The softmax is online in the
 // log2 domain across 128-token tiles.
 //
-// One CTA = one (sequence, KV head, split).  Warp roles:
-//   warp 0      bulk copies of the tile's packed K and V codes into a 4-stage ring
-//   warp 1      TMEM allocation, MMA issue (one thread)
-//   warps 2-5   token warps (thread = token of the tile): unpack K codes to u8 in
-//               tensor memory (A of the score MMA) and V codes to u8 in shared memory
-//               (A of the value MMA, channel-major), then scores, online softmax and
-//               the probability limbs (B of the value MMA)
-//   warps 6-9   channel warps (thread = channel): rescale and accumulate the value
-//               MMA's int32 result into fp32 outputs
+// One CTA = one (sequence, KV head, split), five warps:
+//   warp 0      bulk copies of each tile's packed K and V codes into a 4-stage ring
+//   warps 1-4   token warps.  Thread = token of the tile while widening codes to u8
+//               (K codes into tensor memory as A of the score MMA, V codes into
+//               channel-major shared memory as A of the value MMA) and while turning
+//               scores into probability limbs (B of the value MMA); thread = channel
+//               while accumulating the value MMA's int32 result.  One elected lane
+//               issues the MMAs after a named barrier of the four warps.
+// Per tile i the token warps run: softmax(i) -> value MMA(i); accumulate(i-1);
+// widen(i+1) -> score MMA(i+1), so each MMA has a whole phase to complete before its
+// result is read.  Small CTAs (160 threads, ~72 KB shared memory, 128 TMEM columns)
+// let three run per SM, keeping about 96 KB of code reads in flight per SM.
 // 2- and 4-bit codes are widened to bytes with two logic ops per 4 codes, which
 // permutes channels inside each 16 (8) channel block; the query limbs and the output
 // channels use the same permutation, so the contraction is unchanged.
@@ -41,12 +44,12 @@ namespace {
 using namespace sm100;
 
 constexpr int kTile = 128;
-constexpr int kThreads = 320;
+constexpr int kThreads = 160;
 constexpr int kStages = 4;
 constexpr int kPartialStride = 132;   // m (log2 domain), l, pad, pad, o[128]
-constexpr int kRing = 4;              // per-tile (corr, F) slots shared with the channel warps
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kQScale = 4194303.0f; // 2^22 - 1
+constexpr uint32_t kBarTok = 1;       // named barrier of the four token warps
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int pow2cols(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
@@ -58,16 +61,16 @@ struct Cfg {
   static constexpr int NK = round16(3 * G);                // score MMA N (3 limbs per head)
   static constexpr int NV = round16(2 * G);                // value MMA N (2 limbs per head)
   static constexpr int kColAk = 0;                         // 2 x 32 columns (u8 x 128 channels)
-  static constexpr int kColS = 64;                         // 2 x NK
-  static constexpr int kColO = 64 + 2 * NK;                // 2 x NV
-  static constexpr int kCols = pow2cols(64 + 2 * NK + 2 * NV);
+  static constexpr int kColS = 64;                         // NK
+  static constexpr int kColO = 64 + NK;                    // 2 x NV
+  static constexpr int kCols = pow2cols(64 + NK + 2 * NV);
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int kOffStage = 0;
   static constexpr int kOffAv = (kOffStage + kStages * kStage + 1023) / 1024 * 1024;   // 2 x 16 KB
-  static constexpr int kOffBv = kOffAv + 2 * kTile * 128;                              // 2 x NV rows
+  static constexpr int kOffBv = kOffAv + 2 * kTile * 128;                              // 2 x NV x 128 bytes
   static constexpr int kOffBk = kOffBv + 2 * NV * 128;                                 // NK rows
   static constexpr int kOffMisc = kOffBk + NK * 128;
-  static constexpr int kMiscBytes = 4096;
+  static constexpr int kMiscBytes = 2048;
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
 };
 
@@ -86,15 +89,12 @@ struct DecArgs {
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
-  uint64_t unp_full[2], unp_empty[2], s_full[2], s_empty[2], bv_full[2], o_full[2], o_empty[2];
-  uint64_t red_bar[2], fin_bar, fin_done;
+  uint64_t kdone, vdone[2];
   uint32_t tmem_base;
   int abort;
-  float red[2][4][33];        // per tile parity, per token warp: max s and max (s + log2 scale) per head
-  float qscale[16], qsum[16];
-  float ring_corr[kRing][16], ring_f[kRing][16];
-  float fin_l[16], fin_z[16], fin_m[16];
-  float fin_part[4][2][16];   // per token warp: l and z partial sums
+  float4 red[2][32];          // per parity and value (head maxima), the 4 token warps' partials
+  float c1[16], c2[16];       // per head: qscale * softmax_scale * log2 e, sum(q') * softmax_scale * log2 e
+  float fin[2][16];           // per head: l and z totals
 };
 
 // position p of a widened code row <-> channel
@@ -110,14 +110,11 @@ template <int BITS>
 __device__ __forceinline__ void widen_row(const uint8_t* row, int r, uint32_t (&u)[32]) {
   constexpr int kWords = 4 * BITS;
   uint32_t w[kWords];
+  (void)r;
 #pragma unroll
-  for (int q = 0; q < BITS; ++q) {              // 16-byte pieces, rotated by row to spread banks
-    const int piece = (q + r) % BITS;
-    const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * piece);
-#pragma unroll
-    for (int k = 0; k < BITS; ++k) {
-      if (k == piece) { w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w; }
-    }
+  for (int q = 0; q < BITS; ++q) {
+    const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * q);
+    w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
   }
   if (BITS == 2) {
 #pragma unroll
@@ -164,7 +161,7 @@ __device__ __forceinline__ int kmajor_off(int n, int k) {
 }
 
 template <int BITS, int KIND, int G>
-__global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(DecArgs a) {
+__global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(DecArgs a) {
   using C = Cfg<BITS, G>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,18 +191,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
       mbar_init(&ms->full[s], 1);
       mbar_init(&ms->empty[s], 4);
     }
-    for (int u = 0; u < 2; ++u) {
-      mbar_init(&ms->unp_full[u], 4);
-      mbar_init(&ms->unp_empty[u], 1);
-      mbar_init(&ms->s_full[u], 1);
-      mbar_init(&ms->s_empty[u], 4);
-      mbar_init(&ms->bv_full[u], 4);
-      mbar_init(&ms->o_full[u], 1);
-      mbar_init(&ms->o_empty[u], 4);
-      mbar_init(&ms->red_bar[u], 4);
-    }
-    mbar_init(&ms->fin_bar, 4);
-    mbar_init(&ms->fin_done, 1);
+    mbar_init(&ms->kdone, 1);
+    mbar_init(&ms->vdone[0], 1);
+    mbar_init(&ms->vdone[1], 1);
     ms->abort = 0;
     fence_mbar_init();
   }
@@ -213,29 +201,31 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
     tmem_alloc(&ms->tmem_base, C::kCols);
     tmem_relinquish();
   }
-  if (warp >= 2 && warp < 6) {
+  if (warp >= 1) {
     // query limbs (B of the score MMA): thread = code position p (channel channel_of(p))
-    const int p = threadIdx.x - 64;
+    const int p = threadIdx.x - 32;
     const int c = channel_of<BITS>(p);
     const int wq = p >> 5;
-    float qv[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      qv[h] = a.q[((size_t)b * a.hq + kv * G + h) * kHeadDim + c];
-      float mx = fabsf(qv[h]), sm = qv[h];
+      const float qv = a.q[((size_t)b * a.hq + kv * G + h) * kHeadDim + c];
+      float mx = fabsf(qv), sm = qv;
 #pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        sm += __shfl_xor_sync(0xffffffffu, sm, off);
+      for (int off = 16; off; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+      mx = warp_max(mx);
+      if (lane == 0) {
+        reinterpret_cast<float*>(&ms->red[0][h])[wq] = mx;
+        reinterpret_cast<float*>(&ms->red[1][h])[wq] = sm;
       }
-      if (lane == 0) { ms->red[0][wq][h] = mx; ms->red[1][wq][h] = sm; }
     }
-    named_barrier(1, 128);
+    named_barrier(kBarTok, 128);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
-      const float mx = fmaxf(fmaxf(ms->red[0][0][h], ms->red[0][1][h]), fmaxf(ms->red[0][2][h], ms->red[0][3][h]));
+      const float qv = a.q[((size_t)b * a.hq + kv * G + h) * kHeadDim + c];
+      const float4 m4 = ms->red[0][h];
+      const float mx = fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w));
       const float inv = mx > 0.f ? kQScale / mx : 0.f;
-      const int qi = __float2int_rn(qv[h] * inv);           // |qi| <= 2^22 - 1
+      const int qi = __float2int_rn(qv * inv);              // |qi| <= 2^22 - 1
       const int l0 = (int)(int8_t)(qi & 0xff);
       const int r1 = (qi - l0) >> 8;
       const int l1 = (int)(int8_t)(r1 & 0xff);
@@ -244,8 +234,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
       bk[kmajor_off(G + h, p)] = (uint8_t)l1;
       bk[kmajor_off(2 * G + h, p)] = (uint8_t)l2;
       if (p == 0) {
-        ms->qscale[h] = mx > 0.f ? mx / kQScale : 0.f;
-        ms->qsum[h] = (ms->red[1][0][h] + ms->red[1][1][h]) + (ms->red[1][2][h] + ms->red[1][3][h]);
+        const float4 s4 = ms->red[1][h];
+        ms->c1[h] = (mx > 0.f ? mx / kQScale : 0.f) * a.scale_log2;
+        ms->c2[h] = ((s4.x + s4.y) + (s4.z + s4.w)) * a.scale_log2;
       }
     }
     for (int nrow = 3 * G; nrow < C::NK; ++nrow) bk[kmajor_off(nrow, p)] = 0;
@@ -276,105 +267,98 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
       for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
         mbar_wait(&ms->full[i % kStages], (i / kStages) & 1, &no_abort);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
-      constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 0, 128, C::NV);
-      const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
-      auto value_mma = [&](int j) -> bool {
-        const int u = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&ms->bv_full[u], ph, abort)) return false;
-        if (!mbar_wait(&ms->o_empty[u], ph ^ 1, abort)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + ks * 4096, 16384, 1024, 2);
-          const uint64_t bdesc = desc_kmajor_sw128(bv_addr + u * C::NV * 128 + ks * 32);
-          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, ks > 0);
-        }
-        mma_commit(&ms->o_full[u]);
-        mma_commit(&ms->unp_empty[u]);
-        return true;
-      };
-      bool ok = true;
-      for (int i = 0; i < n && ok; ++i) {
-        const int u = i & 1;
-        const uint32_t ph = (i >> 1) & 1;
-        if (!mbar_wait(&ms->unp_full[u], ph, abort)) break;
-        if (!mbar_wait(&ms->s_empty[u], ph ^ 1, abort)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_i8_ts(tmem + C::kColS + u * C::NK, tmem + C::kColAk + u * 32 + ks * 8,
-                    desc_kmajor_sw128(bk_addr + ks * 32), kIdK, ks > 0);
-        mma_commit(&ms->s_full[u]);
-        if (i >= 1) ok = value_mma(i - 1);
-      }
-      if (ok && n >= 1) value_mma(n - 1);
-    }
-  } else if (warp < 6) {
+  } else {
     // ------------------------------------------------------------- token warps
+    // Every token warp runs the same sequence of named barriers whatever happens; after
+    // a failed (timed-out) wait a warp only skips work, so the barriers always match.
     const int qd = warp & 3;                 // TMEM lane quarter
-    const int r = 32 * qd + lane;            // token row of the tile
-    float m_run[G], l_run[G], z_run[G];
+    const int r = 32 * qd + lane;            // token row while widening / in softmax; channel position while accumulating
+    const bool leader = warp == 1 && lane == 0;
+    bool ok = true;
+    constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
+    constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 1, 128, C::NV);
+    const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
+    float m_run[G], l_run[G], z_run[G], o[G], corr_prev[G], fs_prev[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) { m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; }
+    for (int h = 0; h < G; ++h) {
+      m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; o[h] = 0.f; corr_prev[h] = 0.f; fs_prev[h] = 0.f;
+    }
     uint32_t kmeta_n = 0, vmeta_n = 0, kmeta_c = 0, vmeta_c = 0;
+    float c1[G], c2[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { c1[h] = ms->c1[h]; c2[h] = ms->c2[h]; }
+    const int rx4 = (r & 7) << 4;
 
-    auto unpack = [&](int i) -> bool {
+    // widen tile i's codes: K -> TMEM A (lanes = tokens), V -> channel-major shared A
+    auto widen = [&](int i) {
       const int s = i % kStages;
-      const uint32_t sph = (i / kStages) & 1;
       const int u = i & 1;
-      const uint32_t uph = (i >> 1) & 1;
       const int t = (tile0 + i) * kTile + r;
       if (t < L) {
         kmeta_n = load_meta<KIND>(a.k_meta, pair * a.capacity + t);
         vmeta_n = load_meta<KIND>(a.v_meta, pair * a.capacity + t);
       }
-      if (!mbar_wait(&ms->full[s], sph, abort)) return false;
-      if (!mbar_wait(&ms->unp_empty[u], uph ^ 1, abort)) return false;
-      tc_fence_after();
-      uint32_t wv[32];
-      widen_row<BITS>(stage + s * C::kStage + r * C::kCode, r, wv);
-      tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + C::kColAk + u * 32, wv);
-      widen_row<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, r, wv);
-      uint8_t* arow = av + u * kTile * 128 + r * 128;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / kStages) & 1, abort));
+      if (ok) {
+        uint32_t wv[32];
+        widen_row<BITS>(stage + s * C::kStage + r * C::kCode, r, wv);
+        tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + C::kColAk + u * 32, wv);
+        widen_row<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, r, wv);
+        uint8_t* arow = av + u * kTile * 128 + r * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint4*>(arow + ((j ^ (r & 7)) << 4)) =
-            make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
-      tmem_st_wait();
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&ms->unp_full[u]);
-        mbar_arrive(&ms->empty[s]);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(arow + ((j << 4) ^ rx4)) =
+              make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
+        tmem_st_wait();
       }
-      return true;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->empty[s]);
+      named_barrier(kBarTok, 128);
+      if (leader && ok) {                     // score MMA of tile i
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_i8_ts(tmem + C::kColS, tmem + C::kColAk + u * 32 + ks * 8, desc_kmajor_sw128(bk_addr + ks * 32),
+                    kIdK, ks > 0);
+        mma_commit(&ms->kdone);
+      }
     };
 
-    auto softmax = [&](int i) -> bool {
+    // accumulate the value MMA of tile i into o (thread = channel position r)
+    auto accumulate = [&](int i) {
       const int u = i & 1;
-      const uint32_t ph = (i >> 1) & 1;
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->vdone[u], (i >> 1) & 1, abort));
+      tc_fence_after();
+      uint32_t d[C::NV];
+#pragma unroll
+      for (int c0 = 0; c0 < C::NV; c0 += 16)
+        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColO + u * C::NV + c0,
+                  *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+      tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int di = (int)d[h] + (int)d[G + h] * 256;
+        o[h] = fmaf(o[h], corr_prev[h], fs_prev[h] * (float)di);
+      }
+      tc_fence_before();
+    };
+
+    if (n > 0) widen(0);
+    for (int i = 0; i < n; ++i) {
+      kmeta_c = kmeta_n;
+      vmeta_c = vmeta_n;
+      const int u = i & 1;
       const bool valid = (tile0 + i) * kTile + r < L;
-      if (!mbar_wait(&ms->s_full[u], ph, abort)) return false;
+      // ---- scores of tile i
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->kdone, i & 1, abort));
       tc_fence_after();
       uint32_t d[C::NK];
-      if constexpr (C::NK == 16) {
-        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + u * C::NK, *reinterpret_cast<uint32_t(*)[16]>(d));
-      } else {
 #pragma unroll
-        for (int c0 = 0; c0 < C::NK; c0 += 16)
-          tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + u * C::NK + c0,
-                    *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-      }
+      for (int c0 = 0; c0 < C::NK; c0 += 16)
+        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->s_empty[u]);
       float ks, kz, vs, vz;
       meta_pair<KIND>(kmeta_c, BITS, ks, kz);
       meta_pair<KIND>(vmeta_c, BITS, vs, vz);
@@ -382,75 +366,97 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const int si = (int)d[h] + (int)d[G + h] * 256 + (int)d[2 * G + h] * 65536;
-        const float dot = fmaf(ks, (float)si * ms->qscale[h], kz * ms->qsum[h]);
-        s2[h] = valid ? dot * a.scale_log2 : -CUDART_INF_F;
+        const float dot = fmaf(ks, (float)si * c1[h], kz * c2[h]);
+        s2[h] = valid ? dot : -CUDART_INF_F;
       }
-      // per head, across the 4 token warps: the tile's largest score and the largest
-      // log2 of (probability x value scale) before normalization
+      // ---- tile maxima per head: the largest score and the largest log2(p x value scale)
+      const float lvs = valid && vs > 0.f ? lg2_approx(vs) : -CUDART_INF_F;
       const int par = i & 1;
-      const float lvs = valid && vs > 0.f ? log2f(vs) : -CUDART_INF_F;
 #pragma unroll
-      for (int h = 0; h < 2 * G; ++h) {
-        float v = h < G ? s2[h] : s2[h - G] + lvs;
-#pragma unroll
-        for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        if (lane == 0) ms->red[par][qd][h] = v;
+      for (int h = 0; h < G; ++h) {
+        const float mt = warp_max(s2[h]);
+        const float mu = warp_max(s2[h] + lvs);
+        if (lane == 0) {
+          reinterpret_cast<float*>(&ms->red[par][h])[qd] = mt;
+          reinterpret_cast<float*>(&ms->red[par][G + h])[qd] = mu;
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->red_bar[par]);
-      if (!mbar_wait(&ms->red_bar[par], (i >> 1) & 1, abort)) return false;
+      named_barrier(kBarTok, 128);
       float corr[G], fpt[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float mt = fmaxf(fmaxf(ms->red[par][0][h], ms->red[par][1][h]),
-                               fmaxf(ms->red[par][2][h], ms->red[par][3][h]));
-        const float mu = fmaxf(fmaxf(ms->red[par][0][G + h], ms->red[par][1][G + h]),
-                               fmaxf(ms->red[par][2][G + h], ms->red[par][3][G + h]));
+        const float4 t4 = ms->red[par][h];
+        const float4 u4 = ms->red[par][G + h];
+        const float mt = max3f(t4.x, t4.y, fmaxf(t4.z, t4.w));
+        const float mu = max3f(u4.x, u4.y, fmaxf(u4.z, u4.w));
         const float mn = fmaxf(m_run[h], mt);
-        corr[h] = exp2f(m_run[h] - mn);       // 0 on the first tile
+        corr[h] = ex2_approx(m_run[h] - mn);  // 0 on the first tile
         m_run[h] = mn;
-        // largest p * scale of the tile (slightly widened against log2/exp2 rounding)
-        fpt[h] = exp2f(mu - mn) * 1.000244140625f;
+        fpt[h] = ex2_approx(mu - mn) * 1.000244140625f;   // widened against approximate log2/exp2
       }
-      uint8_t* brow = bv + u * C::NV * 128;
+      // ---- probabilities: l, z in fp32; p x scale as 16-bit limbs (B of the value MMA,
+      // token-major: this token's 2G limb bytes are one 16-byte row, N block of 16 = 2 KB)
+      bool moved = false;
+#pragma unroll
+      for (int h = 0; h < G; ++h) moved |= corr[h] != 1.f;
+      if (moved) {                            // uniform across the CTA: the running max moved
+#pragma unroll
+        for (int h = 0; h < G; ++h) { l_run[h] *= corr[h]; z_run[h] *= corr[h]; }
+      }
+      uint32_t pb[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float p = valid ? exp2f(s2[h] - m_run[h]) : 0.f;
-        l_run[h] = fmaf(l_run[h], corr[h], p);
-        z_run[h] = fmaf(z_run[h], corr[h], p * vz);
-        const float fq = fpt[h] > 0.f ? 65535.0f / fpt[h] : 0.f;
-        const int pi = min(__float2int_rn(p * vs * fq), 65535);
-        brow[kmajor_off(h, r)] = (uint8_t)(pi & 0xff);
-        brow[kmajor_off(G + h, r)] = (uint8_t)(pi >> 8);
+        const float p = valid ? ex2_approx(s2[h] - m_run[h]) : 0.f;
+        l_run[h] += p;
+        z_run[h] = fmaf(p, vz, z_run[h]);
+        const float fq = fpt[h] > 0.f ? __fdividef(65535.0f, fpt[h]) : 0.f;
+        // round to an integer <= 65535 held in the low 16 bits of the float's pattern
+        pb[h] = __float_as_uint(fmaf(p * vs, fq, 12582912.0f));
       }
-      if (threadIdx.x == 64) {
-        const int slot = i % kRing;
+      uint8_t* bcol = bv + u * C::NV * 128 + r * 16;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          ms->ring_corr[slot][h] = corr[h];
-          ms->ring_f[slot][h] = fpt[h] * (1.0f / 65535.0f);
+      for (int nb = 0; nb < C::NV / 16; ++nb) {   // rows 16 nb .. 16 nb + 15 of this token
+        uint32_t wds[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t wv = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int nrow = 16 * nb + 4 * q + e;   // row: limb 0 of heads 0..G-1, then limb 1
+            uint32_t byte = 0;
+            if (nrow < G) byte = pb[nrow] & 0xffu;
+            else if (nrow < 2 * G) byte = (pb[nrow - G] >> 8) & 0xffu;
+            wv |= byte << (8 * e);
+          }
+          wds[q] = wv;
         }
+        *reinterpret_cast<uint4*>(bcol + nb * 2048) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
       }
       fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->bv_full[u]);
-      return true;
-    };
+      tc_fence_before();
+      named_barrier(kBarTok, 128);
+      if (leader && ok) {                     // value MMA of tile i
+        tc_fence_after();
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + kq * 4096, 16384, 1024, 2);
+          const uint64_t bdesc = make_desc(bv_addr + u * C::NV * 128 + kq * 512, 128, 2048, 0);
+          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, kq > 0);
+        }
+        mma_commit(&ms->vdone[u]);
+      }
+      // ---- previous tile's value result, then widen the next tile
+      if (i >= 1) accumulate(i - 1);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        corr_prev[h] = corr[h];
+        fs_prev[h] = fpt[h] * (1.0f / 65535.0f);
+      }
+      if (i + 1 < n) widen(i + 1);
+    }
+    if (n > 0) accumulate(n - 1);
 
-    // zero the padding rows of both value-limb buffers once
-    for (int nrow = 2 * G; nrow < C::NV; ++nrow) {
-      bv[kmajor_off(nrow, r)] = 0;
-      bv[C::NV * 128 + kmajor_off(nrow, r)] = 0;
-    }
-    fence_proxy_async_smem();
-    bool ok = n == 0 || unpack(0);
-    for (int i = 0; i < n && ok; ++i) {
-      kmeta_c = kmeta_n;
-      vmeta_c = vmeta_n;
-      if (i + 1 < n) ok = unpack(i + 1);
-      if (ok) ok = softmax(i);
-    }
-    // per-head totals of l and z over the 128 token threads
+    // ---- split partial: m, l, o + z (z = sum p zero, the same for every channel)
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float l = l_run[h], z = z_run[h];
@@ -459,64 +465,22 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 2 : 1)) decode_tc_kernel(D
         l += __shfl_xor_sync(0xffffffffu, l, off);
         z += __shfl_xor_sync(0xffffffffu, z, off);
       }
-      if (lane == 0) { ms->fin_part[qd][0][h] = l; ms->fin_part[qd][1][h] = z; }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ms->fin_bar);
-    if (threadIdx.x == 64) {
-      if (mbar_wait(&ms->fin_bar, 0, abort)) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          ms->fin_l[h] = (ms->fin_part[0][0][h] + ms->fin_part[1][0][h]) + (ms->fin_part[2][0][h] + ms->fin_part[3][0][h]);
-          ms->fin_z[h] = (ms->fin_part[0][1][h] + ms->fin_part[1][1][h]) + (ms->fin_part[2][1][h] + ms->fin_part[3][1][h]);
-          ms->fin_m[h] = m_run[h];
-        }
-      }
-      mbar_arrive(&ms->fin_done);
-    }
-  } else {
-    // ----------------------------------------------------------- channel warps
-    const int qd = warp & 3;
-    const int mpos = 32 * qd + lane;
-    float o[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) o[h] = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const int u = i & 1;
-      const uint32_t ph = (i >> 1) & 1;
-      if (!mbar_wait(&ms->o_full[u], ph, abort)) break;
-      tc_fence_after();
-      uint32_t d[C::NV];
-#pragma unroll
-      for (int c0 = 0; c0 < C::NV; c0 += 16)
-        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColO + u * C::NV + c0,
-                  *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-      tmem_ld_wait();
-      const int slot = i % kRing;
-      float corr[G], fs[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        corr[h] = ms->ring_corr[slot][h];
-        fs[h] = ms->ring_f[slot][h];
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->o_empty[u]);
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int di = (int)d[h] + ((int)d[G + h] << 8);
-        o[h] = fmaf(o[h], corr[h], fs[h] * (float)di);
+      if (lane == 0) {
+        reinterpret_cast<float*>(&ms->red[0][h])[qd] = l;
+        reinterpret_cast<float*>(&ms->red[0][G + h])[qd] = z;
       }
     }
-    mbar_wait(&ms->fin_done, 0, abort);
-    const int c = channel_of<BITS>(mpos);
+    named_barrier(kBarTok, 128);
+    const int c = channel_of<BITS>(r);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
+      const float4 l4 = ms->red[0][h];
+      const float4 z4 = ms->red[0][G + h];
       float* dst = a.ws + (((size_t)b * a.hq + kv * G + h) * a.num_splits + split) * kPartialStride;
-      dst[4 + c] = o[h] + ms->fin_z[h];
-      if (mpos == 0) {
-        dst[0] = ms->fin_m[h];
-        dst[1] = ms->fin_l[h];
+      dst[4 + c] = o[h] + ((z4.x + z4.y) + (z4.z + z4.w));
+      if (r == 0) {
+        dst[0] = m_run[h];
+        dst[1] = (l4.x + l4.y) + (l4.z + l4.w);
       }
     }
   }
@@ -585,13 +549,14 @@ cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaS
 }  // namespace
 
 // Split count when the caller passes 0: the smallest count whose CTAs fill whole
-// waves of (SMs x 2 resident CTAs) to >= 95%, keeping >= 4 tiles per split; a small
-// problem gets one tile per CTA.
+// waves of (SMs x resident CTAs per SM) to >= 95%, keeping >= 4 tiles per split; a
+// small problem gets one tile per CTA.
 int auto_num_splits(const wushkv_cache& c, int num_q_heads) {
-  (void)num_q_heads;
   const int pairs = c.batch * c.num_kv_heads;
   const int tiles = (c.capacity + kTile - 1) / kTile;
-  const int slots = 2 * num_sms(nullptr);
+  const int g = num_q_heads / c.num_kv_heads;
+  const int per_sm = (g <= 8 && c.qp.bits == 2) ? 3 : 2;
+  const int slots = per_sm * num_sms(nullptr);
   if ((long long)pairs * tiles <= slots) return tiles;
   const int max_s = tiles >= 4 ? tiles / 4 : 1;
   int best = 1;
