@@ -100,25 +100,19 @@ __global__ void __launch_bounds__(kRows) append_rows_kernel(RowArgs a) {
   if (f >= a.total_rows) return;
   SmemRowLoader ld{xs + tid * kPad};
 
-  uint32_t w[4 * BITS];
-  uint16_t m0 = 0, m1 = 0;
-  int32_t flags = 0;
-  if (KIND == WUSHKV_QUEST_INT) {
-    quest_quantize<BITS>(ld, a.alpha, w, m0, flags);
-  } else {
-    affine_quantize<BITS, 3>(ld, a.rank_lo, a.rank_hi, w, m0, m1, flags);
-  }
-
   const int b = f / a.n_new, t = f - b * a.n_new;
   const int pos = __ldg(a.start_pos + b) + t;
-  if (pos < 0 || pos >= a.capacity) {
-    flags |= WUSHKV_STATUS_CAPACITY;
+  const bool store = pos >= 0 && pos < a.capacity;
+  const size_t row = ((size_t)b * a.num_kv_heads + h) * a.capacity + (store ? pos : 0);
+  uint8_t* dst = store ? a.codes + row * (16 * BITS) : nullptr;
+  uint16_t m0 = 0, m1 = 0;
+  int32_t flags = store ? 0 : WUSHKV_STATUS_CAPACITY;
+  if (KIND == WUSHKV_QUEST_INT) {
+    quest_quantize<BITS>(ld, a.alpha, dst, m0, flags);
   } else {
-    const size_t row = ((size_t)b * a.num_kv_heads + h) * a.capacity + pos;
-    uint8_t* dst = a.codes + row * (16 * BITS);
-#pragma unroll
-    for (int q = 0; q < BITS; ++q)
-      st_global_v4(dst + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    affine_quantize<BITS, 3>(ld, a.rank_lo, a.rank_hi, dst, m0, m1, flags);
+  }
+  if (store) {
     if (KIND == WUSHKV_QUEST_INT) {
       a.meta[row] = m0;
     } else {

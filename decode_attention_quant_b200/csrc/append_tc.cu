@@ -11,10 +11,14 @@
 //
 // One persistent CTA per SM, pinned to one KV head (its T_k planes stay in shared
 // memory), walks tiles j, j + C, j + 2C, ... of that head.  Warp roles:
-//   warp 0      TMA producer (K and V tiles, 2-stage rings)
-//   warp 1      TMEM allocation + MMA issue (one thread)
-//   warps 2-5   key epilogue: TMEM -> registers (thread = token row) -> quantize -> store
-//   warps 6-9   value epilogue: shared memory -> registers -> quantize -> store
+//   warp 0       TMA producer (K and V tiles, 2-stage rings)
+//   warp 1       TMEM allocation + MMA issue (one thread)
+//   warps 2-9    key epilogue: TMEM -> registers (thread = token row) -> quantize -> store;
+//                warps 2-5 take the even tiles (accumulator 0), warps 6-9 the odd ones
+//   warps 10-17  value epilogue: shared memory -> registers -> quantize -> store; warps
+//                10-13 take the even tiles (stage 0), 14-17 the odd ones
+// Two tiles are quantized at once, so every scheduler has four epilogue warps to
+// interleave (the quantizer is a long dependent chain per group).
 // Without T_k (identity) the key tiles take the value path and no MMA runs.
 #include "sm100.cuh"
 #include "tmap.h"
@@ -32,7 +36,7 @@ constexpr int kStages = 2;
 constexpr int kBoxBytes = 128 * 128;                 // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kBoxBytes;            // 128 rows x 128 bf16
 constexpr int kPlaneBytes = kTileBytes;              // one bf16 plane of T_k
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;                       // 18 warps
 constexpr int kAccCols = 128;                        // fp32 accumulator columns per buffer
 
 // dynamic shared memory layout (offsets from a 1024-byte aligned base)
@@ -69,6 +73,7 @@ struct Sw128RowLoader {
   const uint8_t* tile;
   int r;
   __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
+    static_assert(kChunk == 32, "loader reads 32 values per chunk");
     const uint8_t* row = tile + (c >> 1) * kBoxBytes + r * 128;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -85,6 +90,7 @@ struct Sw128RowLoader {
 struct TmemRowLoader {
   uint32_t taddr;
   __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
+    static_assert(kChunk == 32, "loader reads 32 values per chunk");
     uint32_t r[32];
     tmem_ld32(taddr + 32 * c, r);
     tmem_ld_wait();
@@ -93,34 +99,36 @@ struct TmemRowLoader {
   }
 };
 
+// Quantize one group (row f of the input, or f < 0 for a row past the end that only
+// joins the warp-collective loads) and write its codes and meta at start_pos[b] + t.
 template <int BITS, int KIND, class Loader>
 __device__ __forceinline__ void quantize_store(Loader& ld, const TcArgs& a, int h, int f, uint8_t* codes,
                                                uint16_t* meta) {
-  uint32_t w[4 * BITS];
-  uint16_t m0 = 0, m1 = 0;
   int32_t flags = 0;
-  if (KIND == WUSHKV_QUEST_INT) {
-    quest_quantize<BITS>(ld, a.alpha, w, m0, flags);
-  } else {
-    affine_quantize<BITS, 3>(ld, a.rank_lo, a.rank_hi, w, m0, m1, flags);
+  size_t row = 0;
+  bool store = false;
+  if (f >= 0) {
+    const int b = f / a.n_new, t = f - b * a.n_new;
+    const int pos = __ldg(a.start_pos + b) + t;
+    store = pos >= 0 && pos < a.capacity;
+    if (!store) flags |= WUSHKV_STATUS_CAPACITY;
+    row = ((size_t)b * a.num_kv_heads + h) * a.capacity + (store ? pos : 0);
   }
-  if (f < 0) return;  // a row past the end that only joined the warp-collective loads
-  const int b = f / a.n_new, t = f - b * a.n_new;
-  const int pos = __ldg(a.start_pos + b) + t;
-  if (pos < 0 || pos >= a.capacity) {
-    flags |= WUSHKV_STATUS_CAPACITY;
+  uint8_t* dst = store ? codes + row * (16 * BITS) : nullptr;
+  uint16_t m0 = 0, m1 = 0;
+  if (KIND == WUSHKV_QUEST_INT) {
+    quest_quantize<BITS>(ld, a.alpha, dst, m0, flags);
   } else {
-    const size_t row = ((size_t)b * a.num_kv_heads + h) * a.capacity + pos;
-    uint8_t* dst = codes + row * (16 * BITS);
-#pragma unroll
-    for (int q = 0; q < BITS; ++q) st_global_v4(dst + 16 * q, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    affine_quantize<BITS, 3>(ld, a.rank_lo, a.rank_hi, dst, m0, m1, flags);
+  }
+  if (store) {
     if (KIND == WUSHKV_QUEST_INT) {
       meta[row] = m0;
     } else {
       reinterpret_cast<uint32_t*>(meta)[row] = (uint32_t)m0 | ((uint32_t)m1 << 16);
     }
   }
-  if (flags) report(a.status, flags);
+  if (flags && f >= 0) report(a.status, flags);
 }
 
 // T_k[h] (fp32, row-major [i][j]) -> three bf16 planes, each laid out as the MMA's B
@@ -130,7 +138,7 @@ __device__ __forceinline__ void quantize_store(Loader& ld, const TcArgs& a, int 
 __device__ __forceinline__ void split_transform(const float* __restrict__ tk, uint8_t* planes, int tid,
                                                 int nthreads) {
   // all of this thread's loads first (independent, so their latencies overlap)
-  constexpr int kMaxPer = 16;
+  constexpr int kMaxPer = kHeadDim * kHeadDim / 4 / (kThreads - 64);
   float4 t4[kMaxPer];
 #pragma unroll
   for (int k = 0; k < kMaxPer; ++k) {
@@ -269,46 +277,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars->acc_full[ab]);
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 10) {
     // --------------------------------------------------------------- key epilogue
+    const int g = (warp - 2) >> 2;            // tile parity this warp group handles
     const int r = 32 * (warp & 3) + lane;     // TMEM lane quarter of this warp
-    for (int li = 0; li < n_loc; ++li) {
+    for (int li = g; li < n_loc; li += 2) {
       const int tile = j0 + li * a.ctas_per_head;
       const int f = tile * kRowsPerTile + r;
+      const uint32_t ph = (li >> 1) & 1;
       if (HAS_T) {
-        const int ab = li & 1;
-        const uint32_t aph = (li >> 1) & 1;
-        if (!mbar_wait(&bars->acc_full[ab], aph, abort)) break;
+        if (!mbar_wait(&bars->acc_full[g], ph, abort)) break;
         tc_fence_after();
-        TmemRowLoader ld{bars->tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + ab * kAccCols};
+        TmemRowLoader ld{bars->tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + g * kAccCols};
         // tcgen05.ld is warp-collective: every lane takes part, rows past the end included
         quantize_store<BITS, KIND>(ld, a, h, f < a.total_rows ? f : -1, a.k_codes, a.k_meta);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
+        if (lane == 0) mbar_arrive(&bars->acc_empty[g]);
       } else {
-        const int s = li % kStages;
-        const uint32_t ph = (li / kStages) & 1;
-        if (!mbar_wait(&bars->full_k[s], ph, abort)) break;
-        Sw128RowLoader ld{kst + s * kTileBytes, r};
+        if (!mbar_wait(&bars->full_k[g], ph, abort)) break;
+        Sw128RowLoader ld{kst + g * kTileBytes, r};
         if (f < a.total_rows) quantize_store<BITS, KIND>(ld, a, h, f, a.k_codes, a.k_meta);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->empty_k[s]);
+        if (lane == 0) mbar_arrive(&bars->empty_k[g]);
       }
     }
   } else {
     // ------------------------------------------------------------- value epilogue
-    const int r = 32 * (warp - 6) + lane;
-    for (int li = 0; li < n_loc; ++li) {
+    const int g = (warp - 10) >> 2;
+    const int r = 32 * ((warp - 10) & 3) + lane;
+    for (int li = g; li < n_loc; li += 2) {
       const int tile = j0 + li * a.ctas_per_head;
-      const int s = li % kStages;
-      const uint32_t ph = (li / kStages) & 1;
-      if (!mbar_wait(&bars->full_v[s], ph, abort)) break;
+      const uint32_t ph = (li >> 1) & 1;
+      if (!mbar_wait(&bars->full_v[g], ph, abort)) break;
       const int f = tile * kRowsPerTile + r;
-      Sw128RowLoader ld{vst + s * kTileBytes, r};
+      Sw128RowLoader ld{vst + g * kTileBytes, r};
       if (f < a.total_rows) quantize_store<BITS, KIND>(ld, a, h, f, a.v_codes, a.v_meta);
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->empty_v[s]);
+      if (lane == 0) mbar_arrive(&bars->empty_v[g]);
     }
   }
 

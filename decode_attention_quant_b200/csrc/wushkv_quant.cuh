@@ -67,24 +67,51 @@ __device__ __forceinline__ double quest_pre(double sumsq, double alpha, int bits
 // The quantizers read a group as four chunks of 32 values through a loader
 // `ld(c, v)` (c = 0..3, v = float[32]): once for the statistics, once for the codes,
 // and again only in the rare exact fallbacks.  Re-reading from shared or tensor
-// memory keeps the register footprint at one chunk.  Loaders may be warp-collective
-// (tensor-memory loads), so every lane of the calling warp runs the same loads: there
-// is no early exit, degenerate groups are handled arithmetically, and the fallbacks
-// run for the whole warp when any lane needs them (exact results are always valid).
+// memory keeps the register footprint at one chunk; each chunk's 32 codes are exactly
+// BITS packed words, written to `dst` (the group's cache row, or nullptr to drop them)
+// as soon as they are known.  Loaders may be warp-collective (tensor-memory loads), so
+// every lane of the calling warp runs the same loads: there is no early exit,
+// degenerate groups are handled arithmetically, and the fallbacks run for the whole
+// warp when any lane needs them (exact results are always valid).
 constexpr int kChunk = 32;
+constexpr int kNumChunks = kHeadDim / kChunk;
+
+template <int BITS>
+__device__ __forceinline__ void store_chunk(uint8_t* dst, int c, const uint32_t (&wc)[BITS]) {
+  if (dst == nullptr) return;
+  uint8_t* p = dst + c * 4 * BITS;
+  if constexpr (BITS == 2) {
+    asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(p), "r"(wc[0]), "r"(wc[1]) : "memory");
+  } else if constexpr (BITS == 4) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(wc[0]), "r"(wc[1]), "r"(wc[2]),
+                 "r"(wc[3])
+                 : "memory");
+  } else {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) reinterpret_cast<uint32_t*>(p)[k] = wc[k];
+  }
+}
+
+// code i (0..31) of a chunk into the chunk's BITS words
+template <int BITS>
+__device__ __forceinline__ void put_chunk_code(uint32_t (&wc)[BITS], int i, uint32_t code) {
+  const int o = BITS * i, wi = o >> 5, sh = o & 31;
+  wc[wi] |= code << sh;
+  if (sh + BITS > 32) wc[wi + 1] |= code >> (32 - sh);
+}
 
 // ---------------------------------------------------------------------------- QuEST
 template <int BITS, class Loader>
-__device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint32_t (&w)[4 * BITS],
-                                               uint16_t& delta_bits, int32_t& flags) {
+__device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t* dst, uint16_t& delta_bits,
+                                               int32_t& flags) {
   constexpr int kHalf = 1 << (BITS - 1);
   constexpr int kMaxCode = (1 << BITS) - 1;
   const unsigned mask = __activemask();
   float s[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) s[k] = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+  for (int c = 0; c < kNumChunks; ++c) {
     float v[kChunk];
     ld(c, v);
 #pragma unroll
@@ -99,7 +126,7 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint32_
   if (__any_sync(mask, ambiguous)) {  // fp64 sum of the exact squares
     double sum = 0.0;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kNumChunks; ++c) {
       float v[kChunk];
       ld(c, v);
 #pragma unroll
@@ -116,34 +143,40 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint32_
   const float inv_up = __fmul_ru(inv, kWidenUp);
   const float m = kMagic + (float)kHalf;
   uint32_t mism = 0u;
-  clear_words<BITS>(w);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+  for (int c = 0; c < kNumChunks; ++c) {
     float v[kChunk];
     ld(c, v);
+    uint32_t wc[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
     for (int i = 0; i < kChunk; ++i) {
       const float y1 = __fmaf_rd(v[i], inv_dn, m);
       const float y2 = __fmaf_rd(v[i], inv_up, m);
       mism |= f2u(y1) ^ f2u(y2);
       const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-      put_code<BITS>(w, c * kChunk + i, (uint32_t)code);
+      put_chunk_code<BITS>(wc, i, (uint32_t)code);
     }
+    store_chunk<BITS>(dst, c, wc);
   }
   if (__any_sync(mask, mism != 0u)) {  // exact: count the thresholds j*Delta (exact in fp32)
-    clear_words<BITS>(w);
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kNumChunks; ++c) {
       float v[kChunk];
       ld(c, v);
+      uint32_t wc[BITS];
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
       for (int i = 0; i < kChunk; ++i) {
         uint32_t code = 0;
 #pragma unroll
         for (int j = -(kHalf - 1); j < kHalf; ++j) code += (v[i] >= (float)j * delta) ? 1u : 0u;
         if (inv == 0.f) code = kHalf;
-        put_code_dyn<BITS>(w, c * kChunk + i, code);
+        put_chunk_code<BITS>(wc, i, code);
       }
+      store_chunk<BITS>(dst, c, wc);
     }
   }
 }
@@ -170,7 +203,7 @@ __device__ __forceinline__ float pick(const float (&a)[KSEL], int idx) {
 }
 
 template <int BITS, int KSEL, class Loader>
-__device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int rank_hi, uint32_t (&w)[4 * BITS],
+__device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int rank_hi, uint8_t* dst,
                                                 uint16_t& scale_bits, uint16_t& zero_bits, int32_t& flags) {
   constexpr int kMaxCode = (1 << BITS) - 1;
   const unsigned mask = __activemask();
@@ -181,8 +214,8 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
     hi_k[k] = __int_as_float(0xff800000);
   }
   float fsum = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+  for (int c = 0; c < kNumChunks; ++c) {
     float v[kChunk];
     ld(c, v);
 #pragma unroll
@@ -205,11 +238,13 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
   uint32_t mism = 0u;
-  clear_words<BITS>(w);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
+#pragma unroll 1
+  for (int c = 0; c < kNumChunks; ++c) {
     float v[kChunk];
     ld(c, v);
+    uint32_t wc[BITS];
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
     for (int i = 0; i < kChunk; ++i) {
       const float d = __fsub_rn(v[i], z);
@@ -217,16 +252,19 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
       const float y2 = __fmaf_rn(d, inv_up, kMagic);
       mism |= f2u(y1) ^ f2u(y2);
       const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-      put_code<BITS>(w, c * kChunk + i, (uint32_t)code);
+      put_chunk_code<BITS>(wc, i, (uint32_t)code);
     }
+    store_chunk<BITS>(dst, c, wc);
   }
   if (__any_sync(mask, mism != 0u)) {  // exact: thresholds zero + (j + 1/2) scale are exact in fp64
-    clear_words<BITS>(w);
     const double zd = (double)z, sd = (double)sc;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < kNumChunks; ++c) {
       float v[kChunk];
       ld(c, v);
+      uint32_t wc[BITS];
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
       for (int i = 0; i < kChunk; ++i) {
         const double xd = (double)v[i];
@@ -237,8 +275,9 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
           code += (xd > t || (xd == t && (j & 1))) ? 1u : 0u;
         }
         if (inv == 0.f) code = 0;
-        put_code_dyn<BITS>(w, c * kChunk + i, code);
+        put_chunk_code<BITS>(wc, i, code);
       }
+      store_chunk<BITS>(dst, c, wc);
     }
   }
 }
