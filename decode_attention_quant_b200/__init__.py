@@ -21,7 +21,7 @@ from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_CAPACITY, STATUS_CT
 HEAD_DIM = 128
 
 __all__ = ["PackedCache", "quantize_append", "transform_query", "decode_attention",
-           "decode_workspace_bytes", "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
+           "decode_attention_noalloc", "decode_workspace_bytes", "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
 
 
 def library():
@@ -152,4 +152,29 @@ def decode_attention(cache: PackedCache, q_t, ctx_len, softmax_scale=None, out=N
                                            _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                            int(num_splits), _ptr(status), _stream(q_t.device, stream))
     _lib.check(rc, "wushkv_decode_attention")
+    return out
+
+
+def decode_attention_noalloc(cache: PackedCache, q_t, ctx_len, softmax_scale=None, out=None, num_splits=0,
+                             status=None, stream=None):
+    """decode_attention with the split partials in the library's fixed scratch array
+    (no workspace is allocated; see wushkv_decode_attention_noalloc for the sharing rules)."""
+    if q_t.dtype != torch.float32 or q_t.dim() != 3 or q_t.shape[0] != cache.batch or q_t.shape[2] != HEAD_DIM \
+            or not q_t.is_contiguous():
+        raise ValueError("q_t must be contiguous float32 [B, Hq, 128]")
+    if ctx_len.dtype != torch.int32 or ctx_len.numel() != cache.batch:
+        raise ValueError("ctx_len must be int32 [B]")
+    hq = int(q_t.shape[1])
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(HEAD_DIM)
+    if out is None:
+        out = torch.empty(q_t.shape, dtype=torch.float32, device=q_t.device)
+    d = cache.desc()
+    rc = library().wushkv_decode_attention_noalloc(ctypes.byref(d), _ptr(q_t), hq, _ptr(ctx_len),
+                                                   float(softmax_scale), _ptr(out), int(num_splits),
+                                                   _ptr(status), _stream(q_t.device, stream))
+    if rc == _lib.ERR_WORKSPACE:
+        raise WushkvError(rc, f"wushkv_decode_attention_noalloc: needs {decode_workspace_bytes(cache, hq, num_splits)} "
+                              f"bytes of scratch, the fixed array holds {_lib.DECODE_STATIC_SCRATCH_BYTES}")
+    _lib.check(rc, "wushkv_decode_attention_noalloc")
     return out

@@ -17,6 +17,9 @@ ERR_MISALIGNED = -3
 ERR_WORKSPACE = -4
 ERR_CUDA = -5
 
+# size of the library's fixed decode scratch array (WUSHKV_DECODE_STATIC_SCRATCH_BYTES)
+DECODE_STATIC_SCRATCH_BYTES = 8 << 20
+
 QUEST_INT = 0
 PCT_AFFINE = 1
 BF16 = 0
@@ -34,6 +37,7 @@ EXPORTS = (
     "wushkv_transform_query",
     "wushkv_decode_workspace_bytes",
     "wushkv_decode_attention",
+    "wushkv_decode_attention_noalloc",
     "wushkv_strerror",
     "wushkv_version",
 )
@@ -78,6 +82,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_decode_workspace_bytes.restype = sz
     lib.wushkv_decode_attention.argtypes = [cp, vp, i32, vp, ctypes.c_float, vp, vp, sz, i32, vp, vp]
     lib.wushkv_decode_attention.restype = ctypes.c_int
+    lib.wushkv_decode_attention_noalloc.argtypes = [cp, vp, i32, vp, ctypes.c_float, vp, i32, vp, vp]
+    lib.wushkv_decode_attention_noalloc.restype = ctypes.c_int
     lib.wushkv_strerror.argtypes = [ctypes.c_int]
     lib.wushkv_strerror.restype = ctypes.c_char_p
     lib.wushkv_version.argtypes = []

@@ -1,6 +1,7 @@
 // C ABI of the WUSH-KV hot path: argument checks on the host, then kernel launches
 // on the caller's stream.  No allocation, no synchronization, no global state
-// besides the per-thread text of the last CUDA error.
+// besides the per-thread text of the last CUDA error.  (The allocation-free decode
+// entry, with its fixed scratch array, is in decode_noalloc.cu.)
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -17,13 +18,19 @@ cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new
 }
 
 namespace {
-
 thread_local char g_cuda_msg[256];
+}  // namespace
 
-int cuda_fail(cudaError_t e) {
+namespace wushkv {
+int record_cuda_error(cudaError_t e) {
   std::snprintf(g_cuda_msg, sizeof(g_cuda_msg), "CUDA error %d: %s", (int)e, cudaGetErrorString(e));
   return WUSHKV_ERR_CUDA;
 }
+}  // namespace wushkv
+
+namespace {
+
+int cuda_fail(cudaError_t e) { return wushkv::record_cuda_error(e); }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

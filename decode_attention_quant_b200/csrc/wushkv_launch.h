@@ -8,6 +8,9 @@
 
 namespace wushkv {
 
+// Stores the text of a CUDA error for wushkv_strerror on this thread; returns WUSHKV_ERR_CUDA.
+int record_cuda_error(cudaError_t e);
+
 cudaError_t launch_quantize_append(const wushkv_cache& c, const void* k_new, const void* v_new,
                                    int in_dtype, int n_new, const int32_t* start_pos,
                                    const float* Tk, int32_t* status, cudaStream_t stream);

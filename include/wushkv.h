@@ -162,6 +162,33 @@ WUSHKV_API int wushkv_decode_attention(const wushkv_cache* cache, const float* q
                             void* workspace, size_t workspace_bytes, int32_t num_splits,
                             int32_t* status, void* stream);
 
+/* Size of the fixed decode scratch array used by wushkv_decode_attention_noalloc:
+ * 8 MiB of device memory per device, enough for the automatic split count of e.g.
+ * batch 32 x 64 query heads at 8K context or batch 16 x 32 heads at 32K. */
+#define WUSHKV_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* wushkv_decode_attention without a workspace argument (an addition of this
+ * library; the method on the pages has no counterpart).  The split partials go to
+ * a fixed array of WUSHKV_DECODE_STATIC_SCRATCH_BYTES in the library's own device
+ * memory, so the call allocates nothing.  It is meant for callers that cannot give
+ * the library scratch memory: a plugin in a host runtime that owns every device
+ * allocation and offers extensions no allocator, or a serving loop that forbids
+ * allocation after start-up to keep its device-memory footprint fixed.
+ *   Arguments, results and errors are those of wushkv_decode_attention, except:
+ *   - WUSHKV_ERR_WORKSPACE when wushkv_decode_workspace_bytes(cache, num_q_heads,
+ *     num_splits) exceeds WUSHKV_DECODE_STATIC_SCRATCH_BYTES (pass a smaller
+ *     num_splits, or use wushkv_decode_attention with a workspace);
+ *   - the first call on each device looks up the array's device address on the
+ *     current device (a CUDA runtime call, no allocation by this library); make that
+ *     first call before any stream capture on that device;
+ *   - every call on a device shares the one array and leaves its partials there;
+ *     nothing in it needs clearing between calls (each call writes every partial it
+ *     reads), but calls that may overlap in time on one device (different streams,
+ *     unordered host threads) race on it and must be serialised by the caller. */
+WUSHKV_API int wushkv_decode_attention_noalloc(const wushkv_cache* cache, const float* q_t,
+                                    int32_t num_q_heads, const int32_t* ctx_len, float softmax_scale,
+                                    float* out, int32_t num_splits, int32_t* status, void* stream);
+
 /* Static text for a wushkv_error code, or the last CUDA error text for WUSHKV_ERR_CUDA
  * on the calling thread. */
 WUSHKV_API const char* wushkv_strerror(int code);
