@@ -15,20 +15,24 @@
 // log2 domain across 128-token tiles.
 //
 // One CTA = one (sequence, KV head, split), five warps:
-//   warp 0      bulk copies of each tile's packed K and V codes into a 4-stage ring
+//   warp 0      one thread: bulk copies of each tile's packed K and V codes into a
+//               4-stage ring, and every MMA, each issued when the mbarrier of the
+//               event it needs completes (tile widened; probabilities written).
 //   warps 1-4   token warps.  Thread = token of the tile while widening codes to u8
 //               (K codes into tensor memory as A of the score MMA, V codes into
 //               channel-major shared memory as A of the value MMA) and while turning
 //               scores into probability limbs (B of the value MMA); thread = channel
-//               while accumulating the value MMA's int32 result.  One elected lane
-//               issues the MMAs after a named barrier of the four warps.
-// Per tile i the token warps run: softmax(i) -> value MMA(i); accumulate(i-1);
-// widen(i+1) -> score MMA(i+1), so each MMA has a whole phase to complete before its
-// result is read.  Small CTAs (160 threads, ~72 KB shared memory, 128 TMEM columns)
-// let three run per SM, keeping about 96 KB of code reads in flight per SM.
-// 2- and 4-bit codes are widened to bytes with two logic ops per 4 codes, which
+//               while accumulating the value MMA's int32 result.  They signal the
+//               issuing thread by mbarrier arrivals and meet each other only to share
+//               each tile's per-head maxima.
+// Per tile i the token warps run: softmax(i) -> [value MMA(i)]; accumulate(i-1);
+// widen(i+1) -> [score MMA(i+1)], so each MMA has a whole phase to complete before
+// its result is read.  Small CTAs (160 threads, ~72 KB shared memory, 128 TMEM
+// columns) let three run per SM, keeping about 96 KB of code reads in flight per SM.
+// 2- and 4-bit key codes are widened to bytes with two logic ops per 4 codes, which
 // permutes channels inside each 16 (8) channel block; the query limbs and the output
-// channels use the same permutation, so the contraction is unchanged.
+// channels use the same permutation, so the contraction is unchanged.  Value codes
+// are widened by masking alone (see widen_row_scaled).
 #include <math_constants.h>
 
 #include <cmath>
@@ -88,13 +92,16 @@ struct DecArgs {
 };
 
 struct Misc {
-  uint64_t full[kStages], empty[kStages];
-  uint64_t kdone, vdone[2];
+  uint64_t full[kStages];     // stage filled (bulk copies)
+  uint64_t kw;                // 4 token warps: tile widened (its stage is free again)
+  uint64_t pr;                // 4 token warps: probabilities of the tile written
+  uint64_t mx;                // 4 token warps: per-warp tile maxima published
+  uint64_t kdone;             // score MMA done
+  uint64_t vdone[2];          // value MMA done, per tile parity
   uint32_t tmem_base;
   int abort;
-  float4 red[2][32];          // per parity and value (head maxima), the 4 token warps' partials
+  float4 red[2][32];          // per tile parity and value (head maxima), the 4 token warps' partials
   float c1[16], c2[16];       // per head: qscale * softmax_scale * log2 e, sum(q') * softmax_scale * log2 e
-  float fin[2][16];           // per head: l and z totals
 };
 
 // position p of a widened code row <-> channel
@@ -107,15 +114,19 @@ __device__ __forceinline__ int channel_of(int p) {
 
 // Packed row (16*BITS bytes at `row`) -> 32 words of four u8 codes (K order as above).
 template <int BITS>
-__device__ __forceinline__ void widen_row(const uint8_t* row, int r, uint32_t (&u)[32]) {
-  constexpr int kWords = 4 * BITS;
-  uint32_t w[kWords];
-  (void)r;
+__device__ __forceinline__ void load_row(const uint8_t* row, uint32_t (&w)[4 * BITS]) {
 #pragma unroll
   for (int q = 0; q < BITS; ++q) {
     const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * q);
     w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
   }
+}
+
+template <int BITS>
+__device__ __forceinline__ void widen_row(const uint8_t* row, uint32_t (&u)[32]) {
+  constexpr int kWords = 4 * BITS;
+  uint32_t w[kWords];
+  load_row<BITS>(row, w);
   if (BITS == 2) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -136,6 +147,38 @@ __device__ __forceinline__ void widen_row(const uint8_t* row, int r, uint32_t (&
       u[g] = (a & 0x00070007u) | ((a & 0x00380038u) << 5);
     }
   }
+}
+
+// Value codes are widened by masking alone: byte p then holds code * value_scale_of(p)
+// (2-bit: 4^((p >> 2) & 3); 4-bit: 16^((p >> 2) & 1); 3-bit: 1).  Position p is an
+// output channel of the value MMA, so the power of two is divided out exactly once,
+// from the split partial.  Largest int32 sum per tile: 65535 * 240 * 128 < 2^31.
+template <int BITS>
+__device__ __forceinline__ void widen_row_scaled(const uint8_t* row, uint32_t (&u)[32]) {
+  if (BITS == 3) {
+    widen_row<BITS>(row, u);
+    return;
+  }
+  uint32_t w[4 * BITS];
+  load_row<BITS>(row, w);
+  if (BITS == 2) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) u[4 * j + k] = w[j] & (0x03030303u << (2 * k));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) u[2 * j + k] = w[j] & (0x0F0F0F0Fu << (4 * k));
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ float value_scale_of(int p) {
+  if (BITS == 2) return (float)(1 << (2 * ((p >> 2) & 3)));
+  if (BITS == 4) return (float)(1 << (4 * ((p >> 2) & 1)));
+  return 1.f;
 }
 
 template <int KIND>
@@ -187,10 +230,10 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
   const size_t pair = (size_t)b * a.hkv + kv;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&ms->full[s], 1);
-      mbar_init(&ms->empty[s], 4);
-    }
+    for (int s = 0; s < kStages; ++s) mbar_init(&ms->full[s], 1);
+    mbar_init(&ms->kw, 4);
+    mbar_init(&ms->pr, 4);
+    mbar_init(&ms->mx, 4);
     mbar_init(&ms->kdone, 1);
     mbar_init(&ms->vdone[0], 1);
     mbar_init(&ms->vdone[1], 1);
@@ -248,13 +291,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
   const uint32_t tmem = ms->tmem_base;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- bulk loads
+    // -------------------------------------------------- bulk loads + MMA issue
+    // One thread, in the order the token warps produce: value MMA(i) once every
+    // token warp has written P(i); score MMA(i+1) once every token warp has widened
+    // tile i+1, which also frees that tile's stage for tile i+1+kStages.
     if (lane == 0) {
+      constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
+      constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 1, 128, C::NV);
+      const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
       int issued = 0;
-      for (int i = 0; i < n; ++i) {
+      auto load = [&](int i) {
         const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&ms->empty[s], ph ^ 1, abort)) break;
         const int t0 = (tile0 + i) * kTile;
         const uint32_t bytes = (uint32_t)min(kTile, L - t0) * C::kCode;
         mbar_arrive_expect_tx(&ms->full[s], 2 * bytes);
@@ -262,22 +309,56 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
         bulk_load(stage + s * C::kStage, a.k_codes + off, bytes, &ms->full[s]);
         bulk_load(stage + s * C::kStage + kTile * C::kCode, a.v_codes + off, bytes, &ms->full[s]);
         ++issued;
+      };
+      auto score_mma = [&](int i) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_i8_ts(tmem + C::kColS, tmem + C::kColAk + (i & 1) * 32 + ks * 8,
+                    desc_kmajor_sw128(bk_addr + ks * 32), kIdK, ks > 0);
+        mma_commit(&ms->kdone);
+      };
+      auto value_mma = [&](int i) {
+        const int u = i & 1;
+        tc_fence_after();
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + kq * 4096, 16384, 1024, 2);
+          const uint64_t bdesc = make_desc(bv_addr + u * C::NV * 128 + kq * 512, 128, 2048, 0);
+          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, kq > 0);
+        }
+        mma_commit(&ms->vdone[u]);
+      };
+      for (int i = 0; i < n && i < kStages; ++i) load(i);
+      bool ok = n > 0 && mbar_wait(&ms->kw, 0, abort);
+      if (ok) {
+        score_mma(0);
+        if (kStages < n) load(kStages);
       }
+      for (int i = 0; ok && i < n; ++i) {
+        if (!(ok = mbar_wait(&ms->pr, i & 1, abort))) break;
+        value_mma(i);
+        if (i + 1 < n) {
+          if (!(ok = mbar_wait(&ms->kw, (i + 1) & 1, abort))) break;
+          score_mma(i + 1);
+          if (i + 1 + kStages < n) load(i + 1 + kStages);
+        }
+      }
+      // no copy may land after the CTA has exited, even after a timeout
       volatile int no_abort = 0;
       for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
         mbar_wait(&ms->full[i % kStages], (i / kStages) & 1, &no_abort);
     }
   } else {
     // ------------------------------------------------------------- token warps
-    // Every token warp runs the same sequence of named barriers whatever happens; after
-    // a failed (timed-out) wait a warp only skips work, so the barriers always match.
+    // Each token warp signals the issuer with one mbarrier arrival per event (tile
+    // widened, probabilities written) and meets the other token warps only to share
+    // each tile's per-head maxima.  After a failed (timed-out) wait a warp skips work
+    // but keeps arriving, so every phase still completes.
     const int qd = warp & 3;                 // TMEM lane quarter
     const int r = 32 * qd + lane;            // token row while widening / in softmax; channel position while accumulating
-    const bool leader = warp == 1 && lane == 0;
+    const uint32_t lanes = (uint32_t)(32 * qd) << 16;
     bool ok = true;
-    constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
-    constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 1, 128, C::NV);
-    const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
     float m_run[G], l_run[G], z_run[G], o[G], corr_prev[G], fs_prev[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -301,9 +382,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / kStages) & 1, abort));
       if (ok) {
         uint32_t wv[32];
-        widen_row<BITS>(stage + s * C::kStage + r * C::kCode, r, wv);
-        tmem_st32(tmem + ((uint32_t)(32 * qd) << 16) + C::kColAk + u * 32, wv);
-        widen_row<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, r, wv);
+        widen_row<BITS>(stage + s * C::kStage + r * C::kCode, wv);
+        tmem_st32(tmem + lanes + C::kColAk + u * 32, wv);
+        widen_row_scaled<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, wv);
         uint8_t* arow = av + u * kTile * 128 + r * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -314,16 +395,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->empty[s]);
-      named_barrier(kBarTok, 128);
-      if (leader && ok) {                     // score MMA of tile i
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_i8_ts(tmem + C::kColS, tmem + C::kColAk + u * 32 + ks * 8, desc_kmajor_sw128(bk_addr + ks * 32),
-                    kIdK, ks > 0);
-        mma_commit(&ms->kdone);
-      }
+      if (lane == 0) mbar_arrive(&ms->kw);
     };
 
     // accumulate the value MMA of tile i into o (thread = channel position r)
@@ -334,8 +406,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       uint32_t d[C::NV];
 #pragma unroll
       for (int c0 = 0; c0 < C::NV; c0 += 16)
-        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColO + u * C::NV + c0,
-                  *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+        tmem_ld16(tmem + lanes + C::kColO + u * C::NV + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
       tmem_ld_wait();
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -357,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       uint32_t d[C::NK];
 #pragma unroll
       for (int c0 = 0; c0 < C::NK; c0 += 16)
-        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + C::kColS + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+        tmem_ld16(tmem + lanes + C::kColS + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
       tmem_ld_wait();
       float ks, kz, vs, vz;
       meta_pair<KIND>(kmeta_c, BITS, ks, kz);
@@ -371,22 +442,23 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       }
       // ---- tile maxima per head: the largest score and the largest log2(p x value scale)
       const float lvs = valid && vs > 0.f ? lg2_approx(vs) : -CUDART_INF_F;
-      const int par = i & 1;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float mt = warp_max(s2[h]);
         const float mu = warp_max(s2[h] + lvs);
         if (lane == 0) {
-          reinterpret_cast<float*>(&ms->red[par][h])[qd] = mt;
-          reinterpret_cast<float*>(&ms->red[par][G + h])[qd] = mu;
+          reinterpret_cast<float*>(&ms->red[u][h])[qd] = mt;
+          reinterpret_cast<float*>(&ms->red[u][G + h])[qd] = mu;
         }
       }
-      named_barrier(kBarTok, 128);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->mx);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->mx, i & 1, abort));
       float corr[G], fpt[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float4 t4 = ms->red[par][h];
-        const float4 u4 = ms->red[par][G + h];
+        const float4 t4 = ms->red[u][h];
+        const float4 u4 = ms->red[u][G + h];
         const float mt = max3f(t4.x, t4.y, fmaxf(t4.z, t4.w));
         const float mu = max3f(u4.x, u4.y, fmaxf(u4.z, u4.w));
         const float mn = fmaxf(m_run[h], mt);
@@ -434,17 +506,8 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(kBarTok, 128);
-      if (leader && ok) {                     // value MMA of tile i
-        tc_fence_after();
-#pragma unroll
-        for (int kq = 0; kq < 4; ++kq) {
-          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + kq * 4096, 16384, 1024, 2);
-          const uint64_t bdesc = make_desc(bv_addr + u * C::NV * 128 + kq * 512, 128, 2048, 0);
-          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, kq > 0);
-        }
-        mma_commit(&ms->vdone[u]);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->pr);
       // ---- previous tile's value result, then widen the next tile
       if (i >= 1) accumulate(i - 1);
 #pragma unroll
@@ -456,7 +519,10 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
     }
     if (n > 0) accumulate(n - 1);
 
-    // ---- split partial: m, l, o + z (z = sum p zero, the same for every channel)
+    // ---- split partial: m, l, o + z (z = sum p zero, the same for every channel).
+    // The widened value codes of channel position r carry a factor value_scale_of(r).
+    named_barrier(kBarTok, 128);              // every token warp is past its last read of red[]
+    const float vfix = 1.0f / value_scale_of<BITS>(r);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float l = l_run[h], z = z_run[h];
@@ -477,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       const float4 l4 = ms->red[0][h];
       const float4 z4 = ms->red[0][G + h];
       float* dst = a.ws + (((size_t)b * a.hq + kv * G + h) * a.num_splits + split) * kPartialStride;
-      dst[4 + c] = o[h] + ((z4.x + z4.y) + (z4.z + z4.w));
+      dst[4 + c] = fmaf(o[h], vfix, (z4.x + z4.y) + (z4.z + z4.w));
       if (r == 0) {
         dst[0] = m_run[h];
         dst[1] = (l4.x + l4.y) + (l4.z + l4.w);
