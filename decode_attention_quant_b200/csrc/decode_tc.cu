@@ -14,21 +14,23 @@
 // (QuEST: scale = Delta, zero = -(2^(b-1) - 1/2) Delta.)  The softmax is online in the
 // log2 domain across 128-token tiles.
 //
-// One CTA = one (sequence, KV head, split), five warps:
+// One CTA = one (sequence, KV head, split); tiles of 256 tokens, five warps:
 //   warp 0      one thread: bulk copies of each tile's packed K and V codes into a
-//               4-stage ring, and every MMA, each issued when the mbarrier of the
-//               event it needs completes (tile widened; probabilities written).
-//   warps 1-4   token warps.  Thread = token of the tile while widening codes to u8
-//               (K codes into tensor memory as A of the score MMA, V codes into
-//               channel-major shared memory as A of the value MMA) and while turning
-//               scores into probability limbs (B of the value MMA); thread = channel
-//               while accumulating the value MMA's int32 result.  They signal the
-//               issuing thread by mbarrier arrivals and meet each other only to share
-//               each tile's per-head maxima.
-// Per tile i the token warps run: softmax(i) -> [value MMA(i)]; accumulate(i-1);
-// widen(i+1) -> [score MMA(i+1)], so each MMA has a whole phase to complete before
-// its result is read.  Small CTAs (160 threads, ~72 KB shared memory, 128 TMEM
-// columns) let three run per SM, keeping about 96 KB of code reads in flight per SM.
+//               ring of stages, and every MMA, each issued when the mbarrier of the
+//               event it needs completes (key codes widened; probabilities written).
+//   warps 1-4   token warps.  Thread = tokens r and 128 + r of the tile (lane r of
+//               the two M = 128 score MMAs) while widening codes to u8 (K codes into
+//               tensor memory as A of the score MMAs, V codes into channel-major
+//               shared memory as A of the value MMAs) and while turning scores into
+//               probability limbs (B of the value MMAs); thread = channel while
+//               accumulating the value MMAs' int32 result.  They signal the issuing
+//               thread by mbarrier arrivals and meet each other only to share each
+//               tile's maxima.
+// Per tile i the token warps run: softmax(i) -> [value MMAs(i)]; widen K(i+1) ->
+// [score MMAs(i+1)]; accumulate(i); widen V(i+1).  Every buffer is single: each is
+// rewritten only after the event that ends its last read.  Two tokens per thread
+// halve the per-tile work (waits, maxima exchange, rescaling, accumulation) per
+// token.  Two CTAs run per SM (up to ~113 KB shared memory, <= 256 TMEM columns).
 // 2- and 4-bit key codes are widened to bytes with two logic ops per 4 codes, which
 // permutes channels inside each 16 (8) channel block; the query limbs and the output
 // channels use the same permutation, so the contraction is unchanged.  Value codes
@@ -47,35 +49,43 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTile = 128;
+constexpr int kHalf = 128;              // tokens of one MMA (M) = one sweep of the 128 TMEM lanes
+constexpr int kTile = 2 * kHalf;        // tokens per pipeline step: two per token-warp thread
 constexpr int kThreads = 160;
-constexpr int kStages = 4;
-constexpr int kPartialStride = 132;   // m (log2 domain), l, pad, pad, o[128]
+constexpr int kPartialStride = 132;     // m (log2 domain), l, pad, pad, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kQScale = 4194303.0f; // 2^22 - 1
-constexpr uint32_t kBarTok = 1;       // named barrier of the four token warps
+constexpr float kQScale = 4194303.0f;   // 2^22 - 1
+constexpr uint32_t kBarTok = 1;         // named barrier of the four token warps
+constexpr int kSmemPerCta = (233472 - 2 * 1024) / 2;   // two CTAs per SM
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int pow2cols(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
+__host__ __device__ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 template <int BITS, int G>
 struct Cfg {
   static constexpr int kCode = 16 * BITS;                  // packed bytes per token row
-  static constexpr int kStage = 2 * kTile * kCode;         // K and V codes of one tile
+  static constexpr int kStage = 2 * kTile * kCode;         // K then V codes of one tile
   static constexpr int NK = round16(3 * G);                // score MMA N (3 limbs per head)
   static constexpr int NV = round16(2 * G);                // value MMA N (2 limbs per head)
-  static constexpr int kColAk = 0;                         // 2 x 32 columns (u8 x 128 channels)
-  static constexpr int kColS = 64;                         // NK
-  static constexpr int kColO = 64 + NK;                    // 2 x NV
-  static constexpr int kCols = pow2cols(64 + NK + 2 * NV);
-  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr int kColAk = 0;                         // 2 halves x 32 columns (u8 x 128 channels)
+  static constexpr int kColS = 64;                         // 2 halves x NK
+  static constexpr int kColO = 64 + 2 * NK;                // NV
+  static constexpr int kCols = pow2cols(64 + 2 * NK + NV);
+  // shared memory (offsets from a 1024-byte aligned base): stages, then the widened V
+  // codes of both halves (channel-major, 128-byte swizzled), the probability limbs of
+  // both halves, the query limbs, barriers and reduction scratch
+  static constexpr int kFixed = 2 * kHalf * 128 + 2 * NV * 128 + NK * 128 + 2048 + 1024;
+  static constexpr int kStages = cmin(4, (kSmemPerCta - kFixed) / kStage);
   static constexpr int kOffStage = 0;
-  static constexpr int kOffAv = (kOffStage + kStages * kStage + 1023) / 1024 * 1024;   // 2 x 16 KB
-  static constexpr int kOffBv = kOffAv + 2 * kTile * 128;                              // 2 x NV x 128 bytes
-  static constexpr int kOffBk = kOffBv + 2 * NV * 128;                                 // NK rows
+  static constexpr int kOffAv = (kOffStage + kStages * kStage + 1023) / 1024 * 1024;
+  static constexpr int kOffBv = kOffAv + 2 * kHalf * 128;
+  static constexpr int kOffBk = kOffBv + 2 * NV * 128;
   static constexpr int kOffMisc = kOffBk + NK * 128;
   static constexpr int kMiscBytes = 2048;
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
+  static_assert(kStages >= 2, "too little shared memory for a double-buffered ring");
+  static_assert(kSmem <= kSmemPerCta, "two CTAs must fit on an SM");
 };
 
 struct DecArgs {
@@ -92,15 +102,15 @@ struct DecArgs {
 };
 
 struct Misc {
-  uint64_t full[kStages];     // stage filled (bulk copies)
-  uint64_t kw;                // 4 token warps: tile widened (its stage is free again)
-  uint64_t pr;                // 4 token warps: probabilities of the tile written
+  uint64_t full[4];           // stage filled (bulk copies)
+  uint64_t kw;                // 4 token warps: key codes of the tile widened
+  uint64_t pr;                // 4 token warps: probabilities written (value codes widened before)
   uint64_t mx;                // 4 token warps: per-warp tile maxima published
-  uint64_t kdone;             // score MMA done
-  uint64_t vdone[2];          // value MMA done, per tile parity
+  uint64_t kdone;             // score MMAs of the tile done
+  uint64_t vdone;             // value MMAs of the tile done
   uint32_t tmem_base;
   int abort;
-  float4 red[2][32];          // per tile parity and value (head maxima), the 4 token warps' partials
+  float4 red[2][33];          // per tile parity: head maxima and the value-scale maximum, per token warp
   float c1[16], c2[16];       // per head: qscale * softmax_scale * log2 e, sum(q') * softmax_scale * log2 e
 };
 
@@ -204,8 +214,9 @@ __device__ __forceinline__ int kmajor_off(int n, int k) {
 }
 
 template <int BITS, int KIND, int G>
-__global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(DecArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecArgs a) {
   using C = Cfg<BITS, G>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage = smem + C::kOffStage;
@@ -230,13 +241,12 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
   const size_t pair = (size_t)b * a.hkv + kv;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&ms->full[s], 1);
+    for (int s = 0; s < S; ++s) mbar_init(&ms->full[s], 1);
     mbar_init(&ms->kw, 4);
     mbar_init(&ms->pr, 4);
     mbar_init(&ms->mx, 4);
     mbar_init(&ms->kdone, 1);
-    mbar_init(&ms->vdone[0], 1);
-    mbar_init(&ms->vdone[1], 1);
+    mbar_init(&ms->vdone, 1);
     ms->abort = 0;
     fence_mbar_init();
   }
@@ -292,16 +302,17 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
 
   if (warp == 0) {
     // -------------------------------------------------- bulk loads + MMA issue
-    // One thread, in the order the token warps produce: value MMA(i) once every
-    // token warp has written P(i); score MMA(i+1) once every token warp has widened
-    // tile i+1, which also frees that tile's stage for tile i+1+kStages.
+    // One thread, in the order the token warps produce: the value MMAs of tile i once
+    // every token warp has written P(i) (its value codes were widened before), which
+    // also frees tile i's stage for tile i + S; the score MMAs of tile i+1 once every
+    // token warp has widened its key codes.
     if (lane == 0) {
       constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
       constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 1, 128, C::NV);
       const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
       int issued = 0;
       auto load = [&](int i) {
-        const int s = i % kStages;
+        const int s = i % S;
         const int t0 = (tile0 + i) * kTile;
         const uint32_t bytes = (uint32_t)min(kTile, L - t0) * C::kCode;
         mbar_arrive_expect_tx(&ms->full[s], 2 * bytes);
@@ -310,214 +321,234 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
         bulk_load(stage + s * C::kStage + kTile * C::kCode, a.v_codes + off, bytes, &ms->full[s]);
         ++issued;
       };
-      auto score_mma = [&](int i) {
+      auto score_mma = [&]() {
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_i8_ts(tmem + C::kColS, tmem + C::kColAk + (i & 1) * 32 + ks * 8,
-                    desc_kmajor_sw128(bk_addr + ks * 32), kIdK, ks > 0);
+        for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_i8_ts(tmem + C::kColS + hb * C::NK, tmem + C::kColAk + hb * 32 + ks * 8,
+                      desc_kmajor_sw128(bk_addr + ks * 32), kIdK, ks > 0);
         mma_commit(&ms->kdone);
       };
-      auto value_mma = [&](int i) {
-        const int u = i & 1;
+      auto value_mma = [&]() {
         tc_fence_after();
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq) {
-          const uint64_t adesc = make_desc(av_addr + u * kTile * 128 + kq * 4096, 16384, 1024, 2);
-          const uint64_t bdesc = make_desc(bv_addr + u * C::NV * 128 + kq * 512, 128, 2048, 0);
-          mma_i8_ss(tmem + C::kColO + u * C::NV, adesc, bdesc, kIdV, kq > 0);
-        }
-        mma_commit(&ms->vdone[u]);
+        for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const uint64_t adesc = make_desc(av_addr + hb * kHalf * 128 + kq * 4096, 16384, 1024, 2);
+            const uint64_t bdesc = make_desc(bv_addr + hb * C::NV * 128 + kq * 512, 128, 2048, 0);
+            mma_i8_ss(tmem + C::kColO, adesc, bdesc, kIdV, (hb | kq) > 0);
+          }
+        mma_commit(&ms->vdone);
       };
-      for (int i = 0; i < n && i < kStages; ++i) load(i);
+      for (int i = 0; i < n && i < S; ++i) load(i);
       bool ok = n > 0 && mbar_wait(&ms->kw, 0, abort);
-      if (ok) {
-        score_mma(0);
-        if (kStages < n) load(kStages);
-      }
+      if (ok) score_mma();
       for (int i = 0; ok && i < n; ++i) {
         if (!(ok = mbar_wait(&ms->pr, i & 1, abort))) break;
-        value_mma(i);
+        value_mma();
+        if (i + S < n) load(i + S);
         if (i + 1 < n) {
           if (!(ok = mbar_wait(&ms->kw, (i + 1) & 1, abort))) break;
-          score_mma(i + 1);
-          if (i + 1 + kStages < n) load(i + 1 + kStages);
+          score_mma();
         }
       }
       // no copy may land after the CTA has exited, even after a timeout
       volatile int no_abort = 0;
-      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_wait(&ms->full[i % kStages], (i / kStages) & 1, &no_abort);
+      for (int i = (issued > S ? issued - S : 0); i < issued; ++i)
+        mbar_wait(&ms->full[i % S], (i / S) & 1, &no_abort);
     }
   } else {
     // ------------------------------------------------------------- token warps
-    // Each token warp signals the issuer with one mbarrier arrival per event (tile
-    // widened, probabilities written) and meets the other token warps only to share
-    // each tile's per-head maxima.  After a failed (timed-out) wait a warp skips work
-    // but keeps arriving, so every phase still completes.
+    // Thread = tokens r and 128 + r of the tile (TMEM lane r of both score halves)
+    // while widening and in the softmax; channel position r while accumulating.
+    // Each token warp signals the issuing thread with one mbarrier arrival per event
+    // and meets the other token warps only to share each tile's maxima.  After a
+    // failed (timed-out) wait a warp skips work but keeps arriving, so every phase
+    // still completes.
     const int qd = warp & 3;                 // TMEM lane quarter
-    const int r = 32 * qd + lane;            // token row while widening / in softmax; channel position while accumulating
+    const int r = 32 * qd + lane;
     const uint32_t lanes = (uint32_t)(32 * qd) << 16;
     bool ok = true;
-    float m_run[G], l_run[G], z_run[G], o[G], corr_prev[G], fs_prev[G];
+    float m_run[G], l_run[G], z_run[G], o[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; o[h] = 0.f; corr_prev[h] = 0.f; fs_prev[h] = 0.f;
-    }
-    uint32_t kmeta_n = 0, vmeta_n = 0, kmeta_c = 0, vmeta_c = 0;
+    for (int h = 0; h < G; ++h) { m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; o[h] = 0.f; }
+    uint32_t kmeta[2] = {0u, 0u}, vmeta[2] = {0u, 0u};
     float c1[G], c2[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { c1[h] = ms->c1[h]; c2[h] = ms->c2[h]; }
     const int rx4 = (r & 7) << 4;
 
-    // widen tile i's codes: K -> TMEM A (lanes = tokens), V -> channel-major shared A
-    auto widen = [&](int i) {
-      const int s = i % kStages;
-      const int u = i & 1;
+    // key codes of tile i -> TMEM A (lane = token), and the tile's meta
+    auto widen_k = [&](int i) {
+      const int s = i % S;
       const int t = (tile0 + i) * kTile + r;
-      if (t < L) {
-        kmeta_n = load_meta<KIND>(a.k_meta, pair * a.capacity + t);
-        vmeta_n = load_meta<KIND>(a.v_meta, pair * a.capacity + t);
-      }
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / kStages) & 1, abort));
-      if (ok) {
-        uint32_t wv[32];
-        widen_row<BITS>(stage + s * C::kStage + r * C::kCode, wv);
-        tmem_st32(tmem + lanes + C::kColAk + u * 32, wv);
-        widen_row_scaled<BITS>(stage + s * C::kStage + kTile * C::kCode + r * C::kCode, wv);
-        uint8_t* arow = av + u * kTile * 128 + r * 128;
+      const size_t mrow = pair * a.capacity + t;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(arow + ((j << 4) ^ rx4)) =
-              make_uint4(wv[4 * j], wv[4 * j + 1], wv[4 * j + 2], wv[4 * j + 3]);
+      for (int j = 0; j < 2; ++j)
+        if (t + kHalf * j < L) {
+          kmeta[j] = load_meta<KIND>(a.k_meta, mrow + kHalf * j);
+          vmeta[j] = load_meta<KIND>(a.v_meta, mrow + kHalf * j);
+        }
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / S) & 1, abort));
+      if (ok) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          uint32_t wv[32];
+          widen_row<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, wv);
+          tmem_st32(tmem + lanes + C::kColAk + 32 * j, wv);
+        }
         tmem_st_wait();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->kw);
     };
-
-    // accumulate the value MMA of tile i into o (thread = channel position r)
-    auto accumulate = [&](int i) {
-      const int u = i & 1;
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->vdone[u], (i >> 1) & 1, abort));
-      tc_fence_after();
-      uint32_t d[C::NV];
+    // value codes of tile i -> channel-major shared A of the value MMA (published by
+    // the arrival on pr after the tile's probabilities)
+    auto widen_v = [&](int i) {
+      const int s = i % S;
+      if (ok) {
 #pragma unroll
-      for (int c0 = 0; c0 < C::NV; c0 += 16)
-        tmem_ld16(tmem + lanes + C::kColO + u * C::NV + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-      tmem_ld_wait();
+        for (int j = 0; j < 2; ++j) {
+          uint32_t wv[32];
+          widen_row_scaled<BITS>(stage + s * C::kStage + kTile * C::kCode + (r + kHalf * j) * C::kCode, wv);
+          uint8_t* arow = av + j * kHalf * 128 + r * 128;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int di = (int)d[h] + (int)d[G + h] * 256;
-        o[h] = fmaf(o[h], corr_prev[h], fs_prev[h] * (float)di);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(arow + ((c << 4) ^ rx4)) =
+                make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        }
       }
-      tc_fence_before();
+      fence_proxy_async_smem();
     };
 
-    if (n > 0) widen(0);
+    if (n > 0) {
+      widen_k(0);
+      widen_v(0);
+    }
     for (int i = 0; i < n; ++i) {
-      kmeta_c = kmeta_n;
-      vmeta_c = vmeta_n;
       const int u = i & 1;
-      const bool valid = (tile0 + i) * kTile + r < L;
-      // ---- scores of tile i
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->kdone, i & 1, abort));
-      tc_fence_after();
-      uint32_t d[C::NK];
+      const int tb = (tile0 + i) * kTile + r;
+      const bool valid[2] = {tb < L, tb + kHalf < L};
+      float ks[2], kz[2], vs[2], vz[2];
 #pragma unroll
-      for (int c0 = 0; c0 < C::NK; c0 += 16)
-        tmem_ld16(tmem + lanes + C::kColS + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-      tmem_ld_wait();
-      float ks, kz, vs, vz;
-      meta_pair<KIND>(kmeta_c, BITS, ks, kz);
-      meta_pair<KIND>(vmeta_c, BITS, vs, vz);
-      float s2[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const int si = (int)d[h] + (int)d[G + h] * 256 + (int)d[2 * G + h] * 65536;
-        const float dot = fmaf(ks, (float)si * c1[h], kz * c2[h]);
-        s2[h] = valid ? dot : -CUDART_INF_F;
+      for (int j = 0; j < 2; ++j) {
+        meta_pair<KIND>(kmeta[j], BITS, ks[j], kz[j]);
+        meta_pair<KIND>(vmeta[j], BITS, vs[j], vz[j]);
+        if (!valid[j]) vs[j] = 0.f;
       }
-      // ---- tile maxima per head: the largest score and the largest log2(p x value scale)
-      const float lvs = valid && vs > 0.f ? lg2_approx(vs) : -CUDART_INF_F;
+      // ---- scores of tile i (both halves)
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->kdone, u, abort));
+      tc_fence_after();
+      float s2[2][G];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        uint32_t d[C::NK];
+#pragma unroll
+        for (int c0 = 0; c0 < C::NK; c0 += 16)
+          tmem_ld16(tmem + lanes + C::kColS + j * C::NK + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const int si = (int)d[h] + (int)d[G + h] * 256 + (int)d[2 * G + h] * 65536;
+          const float dot = fmaf(ks[j], (float)si * c1[h], kz[j] * c2[h]);
+          s2[j][h] = valid[j] ? dot : -CUDART_INF_F;
+        }
+      }
+      // ---- tile maxima: per head the largest score; the largest value scale
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float mt = warp_max(s2[h]);
-        const float mu = warp_max(s2[h] + lvs);
-        if (lane == 0) {
-          reinterpret_cast<float*>(&ms->red[u][h])[qd] = mt;
-          reinterpret_cast<float*>(&ms->red[u][G + h])[qd] = mu;
-        }
+        const float mt = warp_max(fmaxf(s2[0][h], s2[1][h]));
+        if (lane == 0) reinterpret_cast<float*>(&ms->red[u][h])[qd] = mt;
+      }
+      {
+        const float vm = warp_max(fmaxf(vs[0], vs[1]));
+        if (lane == 0) reinterpret_cast<float*>(&ms->red[u][32])[qd] = vm;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->mx);
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->mx, i & 1, abort));
-      float corr[G], fpt[G];
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->mx, u, abort));
+      const float4 v4 = ms->red[u][32];
+      // widened against approximate exp2, so that every p * scale stays below F
+      const float vmax = max3f(v4.x, v4.y, fmaxf(v4.z, v4.w)) * 1.000244140625f;
+      float corr[G], fq[G], fs[G];
+      bool moved = false;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float4 t4 = ms->red[u][h];
-        const float4 u4 = ms->red[u][G + h];
         const float mt = max3f(t4.x, t4.y, fmaxf(t4.z, t4.w));
-        const float mu = max3f(u4.x, u4.y, fmaxf(u4.z, u4.w));
         const float mn = fmaxf(m_run[h], mt);
         corr[h] = ex2_approx(m_run[h] - mn);  // 0 on the first tile
+        moved |= corr[h] != 1.f;
         m_run[h] = mn;
-        fpt[h] = ex2_approx(mu - mn) * 1.000244140625f;   // widened against approximate log2/exp2
+        // F = 2^(mt - m) * (largest value scale) bounds every p * scale of the tile
+        const float f = ex2_approx(mt - mn) * vmax;
+        fq[h] = f > 0.f ? __fdividef(65535.0f, f) : 0.f;
+        fs[h] = f * (1.0f / 65535.0f);
       }
-      // ---- probabilities: l, z in fp32; p x scale as 16-bit limbs (B of the value MMA,
-      // token-major: this token's 2G limb bytes are one 16-byte row, N block of 16 = 2 KB)
-      bool moved = false;
-#pragma unroll
-      for (int h = 0; h < G; ++h) moved |= corr[h] != 1.f;
-      if (moved) {                            // uniform across the CTA: the running max moved
+      if (moved) {                            // uniform across the CTA: a running max moved
 #pragma unroll
         for (int h = 0; h < G; ++h) { l_run[h] *= corr[h]; z_run[h] *= corr[h]; }
       }
-      uint32_t pb[G];
+      // ---- probabilities: l, z in fp32; p x scale as 16-bit limbs (B of the value MMA,
+      // token-major: a token's 2G limb bytes are one 16-byte row, N block of 16 = 2 KB)
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float p = valid ? ex2_approx(s2[h] - m_run[h]) : 0.f;
-        l_run[h] += p;
-        z_run[h] = fmaf(p, vz, z_run[h]);
-        const float fq = fpt[h] > 0.f ? __fdividef(65535.0f, fpt[h]) : 0.f;
-        // round to an integer <= 65535 held in the low 16 bits of the float's pattern
-        pb[h] = __float_as_uint(fmaf(p * vs, fq, 12582912.0f));
-      }
-      uint8_t* bcol = bv + u * C::NV * 128 + r * 16;
+      for (int j = 0; j < 2; ++j) {
+        uint32_t pb[G];
 #pragma unroll
-      for (int nb = 0; nb < C::NV / 16; ++nb) {   // rows 16 nb .. 16 nb + 15 of this token
-        uint32_t wds[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t wv = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int nrow = 16 * nb + 4 * q + e;   // row: limb 0 of heads 0..G-1, then limb 1
-            uint32_t byte = 0;
-            if (nrow < G) byte = pb[nrow] & 0xffu;
-            else if (nrow < 2 * G) byte = (pb[nrow - G] >> 8) & 0xffu;
-            wv |= byte << (8 * e);
-          }
-          wds[q] = wv;
+        for (int h = 0; h < G; ++h) {
+          const float p = valid[j] ? ex2_approx(s2[j][h] - m_run[h]) : 0.f;
+          l_run[h] += p;
+          z_run[h] = fmaf(p, vz[j], z_run[h]);
+          // round to an integer <= 65535 held in the low 16 bits of the float's pattern
+          pb[h] = __float_as_uint(fmaf(p * vs[j], fq[h], 12582912.0f));
         }
-        *reinterpret_cast<uint4*>(bcol + nb * 2048) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        uint8_t* bcol = bv + j * C::NV * 128 + r * 16;
+#pragma unroll
+        for (int nb = 0; nb < C::NV / 16; ++nb) {   // rows 16 nb .. 16 nb + 15 of this token
+          uint32_t wds[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int nrow = 16 * nb + 4 * q + e;   // row: limb 0 of heads 0..G-1, then limb 1
+              uint32_t byte = 0;
+              if (nrow < G) byte = pb[nrow] & 0xffu;
+              else if (nrow < 2 * G) byte = (pb[nrow - G] >> 8) & 0xffu;
+              wv |= byte << (8 * e);
+            }
+            wds[q] = wv;
+          }
+          *reinterpret_cast<uint4*>(bcol + nb * 2048) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->pr);
-      // ---- previous tile's value result, then widen the next tile
-      if (i >= 1) accumulate(i - 1);
+      // ---- next tile's key codes, this tile's value result, next tile's value codes
+      if (i + 1 < n) widen_k(i + 1);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->vdone, u, abort));
+      tc_fence_after();
+      {
+        uint32_t d[C::NV];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        corr_prev[h] = corr[h];
-        fs_prev[h] = fpt[h] * (1.0f / 65535.0f);
+        for (int c0 = 0; c0 < C::NV; c0 += 16)
+          tmem_ld16(tmem + lanes + C::kColO + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const int di = (int)d[h] + (int)d[G + h] * 256;
+          o[h] = fmaf(o[h], corr[h], fs[h] * (float)di);
+        }
       }
-      if (i + 1 < n) widen(i + 1);
+      tc_fence_before();
+      if (i + 1 < n) widen_v(i + 1);
     }
-    if (n > 0) accumulate(n - 1);
 
     // ---- split partial: m, l, o + z (z = sum p zero, the same for every channel).
     // The widened value codes of channel position r carry a factor value_scale_of(r).
@@ -533,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
       }
       if (lane == 0) {
         reinterpret_cast<float*>(&ms->red[0][h])[qd] = l;
-        reinterpret_cast<float*>(&ms->red[0][G + h])[qd] = z;
+        reinterpret_cast<float*>(&ms->red[1][h])[qd] = z;
       }
     }
     named_barrier(kBarTok, 128);
@@ -541,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, (G <= 8 ? 3 : 2)) decode_tc_kernel(D
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float4 l4 = ms->red[0][h];
-      const float4 z4 = ms->red[0][G + h];
+      const float4 z4 = ms->red[1][h];
       float* dst = a.ws + (((size_t)b * a.hq + kv * G + h) * a.num_splits + split) * kPartialStride;
       dst[4 + c] = fmaf(o[h], vfix, (z4.x + z4.y) + (z4.z + z4.w));
       if (r == 0) {
@@ -614,24 +645,20 @@ cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaS
 
 }  // namespace
 
-// Split count when the caller passes 0: the smallest count whose CTAs fill whole
-// waves of (SMs x resident CTAs per SM) to >= 95%, keeping >= 4 tiles per split; a
-// small problem gets one tile per CTA.
+// Split count when the caller passes 0.  Time is modelled as (waves of CTAs over
+// SMs x 2 resident CTAs) x (tiles per split + 1, the +1 for a CTA's set-up and its
+// partial); the count with the least modelled time wins, the smaller on ties.
 int auto_num_splits(const wushkv_cache& c, int num_q_heads) {
-  const int pairs = c.batch * c.num_kv_heads;
+  (void)num_q_heads;
+  const long long pairs = (long long)c.batch * c.num_kv_heads;
   const int tiles = (c.capacity + kTile - 1) / kTile;
-  const int g = num_q_heads / c.num_kv_heads;
-  const int per_sm = (g <= 8 && c.qp.bits == 2) ? 3 : 2;
-  const int slots = per_sm * num_sms(nullptr);
-  if ((long long)pairs * tiles <= slots) return tiles;
-  const int max_s = tiles >= 4 ? tiles / 4 : 1;
+  const long long slots = 2LL * num_sms(nullptr);
   int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= max_s && s <= 256; ++s) {
-    const double w = (double)pairs * s / slots;
-    const double eff = w / std::ceil(w);
-    if (eff >= 0.95) return s;
-    if (eff > best_eff + 1e-9) { best_eff = eff; best = s; }
+  long long best_cost = -1;
+  for (int s = 1; s <= tiles && s <= 256; ++s) {
+    const long long waves = (pairs * s + slots - 1) / slots;
+    const long long cost = waves * ((tiles + s - 1) / s + 1);
+    if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
   }
   return best;
 }
