@@ -30,7 +30,8 @@
 // [score MMAs(i+1)]; accumulate(i); widen V(i+1).  Every buffer is single: each is
 // rewritten only after the event that ends its last read.  Two tokens per thread
 // halve the per-tile work (waits, maxima exchange, rescaling, accumulation) per
-// token.  Two CTAs run per SM (up to ~113 KB shared memory, <= 256 TMEM columns).
+// token.  Up to three CTAs run per SM (2-bit codes, g <= 8: two stages, ~73 KB shared
+// memory and 128 TMEM columns each); wider codes or groups run two.
 // 2- and 4-bit key codes are widened to bytes with two logic ops per 4 codes, which
 // permutes channels inside each 16 (8) channel block; the query limbs and the output
 // channels use the same permutation, so the contraction is unchanged.  Value codes
@@ -56,7 +57,7 @@ constexpr int kPartialStride = 132;     // m (log2 domain), l, pad, pad, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kQScale = 4194303.0f;   // 2^22 - 1
 constexpr uint32_t kBarTok = 1;         // named barrier of the four token warps
-constexpr int kSmemPerCta = (233472 - 2 * 1024) / 2;   // two CTAs per SM
+constexpr int kSmemPerSm = 233472;      // bytes of shared memory per SM, 1 KB of it reserved per CTA
 
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ constexpr int pow2cols(int x) { return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512; }
@@ -76,7 +77,11 @@ struct Cfg {
   // codes of both halves (channel-major, 128-byte swizzled), the probability limbs of
   // both halves, the query limbs, barriers and reduction scratch
   static constexpr int kFixed = 2 * kHalf * 128 + 2 * NV * 128 + NK * 128 + 2048 + 1024;
-  static constexpr int kStages = cmin(4, (kSmemPerCta - kFixed) / kStage);
+  // as many resident CTAs per SM (up to 3) as leave room for a double-buffered ring
+  static constexpr int ring(int ctas) { return (kSmemPerSm / ctas - 1024 - kFixed) / kStage; }
+  static constexpr int kCtas = ring(3) >= 2 ? 3 : 2;
+  static constexpr int kSmemPerCta = kSmemPerSm / kCtas - 1024;
+  static constexpr int kStages = cmin(4, ring(kCtas));
   static constexpr int kOffStage = 0;
   static constexpr int kOffAv = (kOffStage + kStages * kStage + 1023) / 1024 * 1024;
   static constexpr int kOffBv = kOffAv + 2 * kHalf * 128;
@@ -85,7 +90,7 @@ struct Cfg {
   static constexpr int kMiscBytes = 2048;
   static constexpr int kSmem = kOffMisc + kMiscBytes + 1024;
   static_assert(kStages >= 2, "too little shared memory for a double-buffered ring");
-  static_assert(kSmem <= kSmemPerCta, "two CTAs must fit on an SM");
+  static_assert(kSmem <= kSmemPerCta, "the CTAs must fit on an SM");
 };
 
 struct DecArgs {
@@ -214,7 +219,7 @@ __device__ __forceinline__ int kmajor_off(int n, int k) {
 }
 
 template <int BITS, int KIND, int G>
-__global__ void __launch_bounds__(kThreads, 2) decode_tc_kernel(DecArgs a) {
+__global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kernel(DecArgs a) {
   using C = Cfg<BITS, G>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -643,16 +648,24 @@ cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaS
   return launch_kind<BITS, WUSHKV_PCT_AFFINE>(a, batch, out, stream);
 }
 
+// Resident decode CTAs per SM for a cache's bit width and group size (Cfg::kCtas).
+int ctas_per_sm(int bits, int g) {
+  static_assert(Cfg<2, 8>::kCtas == 3 && Cfg<2, 16>::kCtas == 2 && Cfg<3, 1>::kCtas == 2 &&
+                    Cfg<4, 1>::kCtas == 2 && Cfg<4, 16>::kCtas == 2,
+                "keep ctas_per_sm in step with Cfg");
+  return (bits == 2 && g <= 8) ? 3 : 2;
+}
+
 }  // namespace
 
 // Split count when the caller passes 0.  Time is modelled as (waves of CTAs over
-// SMs x 2 resident CTAs) x (tiles per split + 1, the +1 for a CTA's set-up and its
+// SMs x resident CTAs per SM) x (tiles per split + 1, the +1 for a CTA's set-up and its
 // partial); the count with the least modelled time wins, the smaller on ties.
 int auto_num_splits(const wushkv_cache& c, int num_q_heads) {
-  (void)num_q_heads;
   const long long pairs = (long long)c.batch * c.num_kv_heads;
   const int tiles = (c.capacity + kTile - 1) / kTile;
-  const long long slots = 2LL * num_sms(nullptr);
+  const int g = num_q_heads / c.num_kv_heads;
+  const long long slots = (long long)ctas_per_sm(c.qp.bits, g) * num_sms(nullptr);
   int best = 1;
   long long best_cost = -1;
   for (int s = 1; s <= tiles && s <= 256; ++s) {
