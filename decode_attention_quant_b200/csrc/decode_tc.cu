@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       for (int j = 0; j < 2; ++j) {
         meta_pair<KIND>(kmeta[j], BITS, ks[j], kz[j]);
         meta_pair<KIND>(vmeta[j], BITS, vs[j], vz[j]);
-        if (!valid[j]) vs[j] = 0.f;
+        if (!valid[j]) { vs[j] = 0.f; vz[j] = 0.f; }
       }
       // ---- scores of tile i (both halves)
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->kdone, u, abort));
@@ -477,39 +477,36 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       if (lane == 0) mbar_arrive(&ms->mx);
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->mx, u, abort));
       const float4 v4 = ms->red[u][32];
-      // widened against approximate exp2, so that every p * scale stays below F
-      const float vmax = max3f(v4.x, v4.y, fmaxf(v4.z, v4.w)) * 1.000244140625f;
-      float corr[G], fq[G], fs[G];
-      bool moved = false;
+      const float vmax = max3f(v4.x, v4.y, fmaxf(v4.z, v4.w));
+      // limb scale: e * scale * vq <= 65520 (1 + 2^-21) < 65536 for e = 2^(s - mt) <= 1
+      const float vq = vmax > 0.f ? __fdividef(65520.0f, vmax) : 0.f;
+      float corr[G], ch[G], mt[G], lt[G], zt[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float4 t4 = ms->red[u][h];
-        const float mt = max3f(t4.x, t4.y, fmaxf(t4.z, t4.w));
-        const float mn = fmaxf(m_run[h], mt);
+        mt[h] = max3f(t4.x, t4.y, fmaxf(t4.z, t4.w));
+        const float mn = fmaxf(m_run[h], mt[h]);
         corr[h] = ex2_approx(m_run[h] - mn);  // 0 on the first tile
-        moved |= corr[h] != 1.f;
+        ch[h] = ex2_approx(mt[h] - mn);
         m_run[h] = mn;
-        // F = 2^(mt - m) * (largest value scale) bounds every p * scale of the tile
-        const float f = ex2_approx(mt - mn) * vmax;
-        fq[h] = f > 0.f ? __fdividef(65535.0f, f) : 0.f;
-        fs[h] = f * (1.0f / 65535.0f);
+        lt[h] = 0.f;
+        zt[h] = 0.f;
       }
-      if (moved) {                            // uniform across the CTA: a running max moved
-#pragma unroll
-        for (int h = 0; h < G; ++h) { l_run[h] *= corr[h]; z_run[h] *= corr[h]; }
-      }
-      // ---- probabilities: l, z in fp32; p x scale as 16-bit limbs (B of the value MMA,
-      // token-major: a token's 2G limb bytes are one 16-byte row, N block of 16 = 2 KB)
+      // ---- probabilities relative to the tile maximum, e = 2^(s - mt) (p = ch e): sums
+      // in fp32; e x scale as 16-bit limbs (B of the value MMA, token-major: a token's 2G
+      // limb bytes are one 16-byte row, N block of 16 = 2 KB).  Rows past the context
+      // have s = -inf, so e = 0.
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
+        const float vsq = vs[j] * vq;
         uint32_t pb[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float p = valid[j] ? ex2_approx(s2[j][h] - m_run[h]) : 0.f;
-          l_run[h] += p;
-          z_run[h] = fmaf(p, vz[j], z_run[h]);
+          const float e = ex2_approx(s2[j][h] - mt[h]);
+          lt[h] += e;
+          zt[h] = fmaf(e, vz[j], zt[h]);
           // round to an integer <= 65535 held in the low 16 bits of the float's pattern
-          pb[h] = __float_as_uint(fmaf(p * vs[j], fq[h], 12582912.0f));
+          pb[h] = __float_as_uint(fmaf(e, vsq, 12582912.0f));
         }
         uint8_t* bcol = bv + j * C::NV * 128 + r * 16;
 #pragma unroll
@@ -535,6 +532,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->pr);
+      float fs[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        l_run[h] = fmaf(l_run[h], corr[h], ch[h] * lt[h]);
+        z_run[h] = fmaf(z_run[h], corr[h], ch[h] * zt[h]);
+        fs[h] = ch[h] * vmax * (1.0f / 65520.0f);
+      }
       // ---- next tile's key codes, this tile's value result, next tile's value codes
       if (i + 1 < n) widen_k(i + 1);
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->vdone, u, abort));
