@@ -252,6 +252,7 @@ def run_ours(args, rank, world, local):
     if True:
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("timed_steps")       # lets a profiler select these launches
         t0.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
@@ -262,6 +263,7 @@ def run_ours(args, rank, world, local):
             dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
             ev[i][3].record(stream)
         t1.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
     timed_to = time.time()
     clk.__exit__(None, None, None)
@@ -351,9 +353,11 @@ def bench_append(dq, device, args, world):
         flush.zero_()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("append_chunk")      # lets a profiler select these launches
         a.record(stream)
         dq.quantize_append(cache, k, v, sp, tk)
         b.record(stream)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
     ms = max_over_ranks(statistics.median(times), world)

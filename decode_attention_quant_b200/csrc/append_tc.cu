@@ -70,6 +70,7 @@ struct Bars {
 // Row r of a 128-row tile held as two 128B-swizzled boxes of 64 bf16: chunk c of 32
 // values lives in box c / 2, 16-byte pieces 4 (c & 1) .. 4 (c & 1) + 3, swizzled by r & 7.
 struct Sw128RowLoader {
+  static constexpr bool kBf16Exact = true;    // every value is a bf16 input
   const uint8_t* tile;
   int r;
   __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
@@ -88,6 +89,7 @@ struct Sw128RowLoader {
 
 // The fp32 accumulator row of this thread's TMEM lane: chunk c = columns 32c .. 32c+31.
 struct TmemRowLoader {
+  static constexpr bool kBf16Exact = false;   // fp32 transform results
   uint32_t taddr;
   __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
     static_assert(kChunk == 32, "loader reads 32 values per chunk");

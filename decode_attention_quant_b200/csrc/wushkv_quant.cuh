@@ -15,6 +15,12 @@
 //   * codes: the quotient is evaluated with the reciprocal widened by 2^-20 on both
 //     sides; where the two roundings differ the group's codes are recomputed by
 //     exact threshold comparisons (fp32 for QuEST, fp64 for affine thresholds).
+//   * QuEST codes of bf16 inputs (loaders with kBf16Exact) need no bracket: a bf16
+//     value (8 significant bits) and a threshold j*Delta (fp16 step times a small
+//     integer, <= 15 significant bits) are either equal or at least 2^-16 apart
+//     relative to the threshold, far outside the 2^-20 widening.  So one
+//     round-down product with the reciprocal widened away from zero's side (up for
+//     x >= 0, down for x < 0) lands on the exact floor, ties included.
 #pragma once
 #include "wushkv_common.cuh"
 
@@ -142,6 +148,24 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
   const float m = kMagic + (float)kHalf;
+  if constexpr (Loader::kBf16Exact) {
+#pragma unroll 1
+    for (int c = 0; c < kNumChunks; ++c) {
+      float v[kChunk];
+      ld(c, v);
+      uint32_t wc[BITS];
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) wc[k] = 0u;
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) {
+        const float y = __fmaf_rd(v[i], v[i] < 0.f ? inv_dn : inv_up, m);
+        const int32_t code = min(max(f2i(y) - kMagicBits, 0), kMaxCode);
+        put_chunk_code<BITS>(wc, i, (uint32_t)code);
+      }
+      store_chunk<BITS>(dst, c, wc);
+    }
+    return;
+  }
   uint32_t mism = 0u;
 #pragma unroll 1
   for (int c = 0; c < kNumChunks; ++c) {
@@ -284,6 +308,7 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
 
 // Loader over a group held in a shared-memory row of fp32 values.
 struct SmemRowLoader {
+  static constexpr bool kBf16Exact = false;   // fp32 rows: any value
   const float* row;
   __device__ __forceinline__ void operator()(int c, float (&v)[kChunk]) const {
 #pragma unroll

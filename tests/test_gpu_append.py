@@ -183,3 +183,49 @@ def test_append_identity_transform_equals_no_transform():
     torch.cuda.synchronize()
     for name, t in a.tensors().items():
         assert torch.equal(t, b.tensors()[name]), name
+
+
+def _bf16_groups_on_thresholds(n_groups, bits, seed):
+    """bf16 value groups whose QuEST step Delta has <= 8 significant bits and which
+    hold elements exactly on thresholds j*Delta (found by a seeded search, oracle side:
+    each threshold replaces the element nearest to it, so Delta barely moves)."""
+    rng = np.random.default_rng(seed)
+    alpha = QUEST_ALPHA[bits]
+    half = 1 << (bits - 1)
+    out = []
+    for _ in range(200 * n_groups):
+        if len(out) == n_groups:
+            break
+        g = torch.from_numpy(rng.standard_normal(128).astype(np.float32)).bfloat16().float().numpy()
+        d = float(orc.quest_meta(g.astype(np.float64), bits, alpha))
+        mant = np.frexp(d)[0] * 2 ** 8
+        if d == 0 or mant != np.round(mant):          # Delta must be a bf16 value
+            continue
+        for j in range(-(half - 1), half):
+            t = np.float32(j * d)
+            if float(torch.tensor([t]).bfloat16().float()[0]) == t:   # only bf16 thresholds
+                g[np.argmin(np.abs(g - t))] = t
+        if float(orc.quest_meta(g.astype(np.float64), bits, alpha)) == d:
+            out.append(g)
+    assert len(out) == n_groups
+    return np.stack(out)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_bf16_values_on_thresholds_bitexact(bits):
+    """Values (bf16, no transform) lying exactly on decision thresholds j*Delta take the
+    single-product path of the tensor-core append; codes must equal the oracle's."""
+    bsz, n, hkv = 1, 256, 1
+    v = _bf16_groups_on_thresholds(n, bits, seed=90 + bits).reshape(bsz, n, hkv, 128)
+    d = orc.fp16_value(np.array([orc.fp16_bits(orc.quest_meta(g.astype(np.float64), bits, QUEST_ALPHA[bits]))
+                                 for g in v.reshape(-1, 128)]))
+    ties = sum(int(np.isin(g, [j * dd for j in range(-(1 << (bits - 1)), 1 << (bits - 1))]).sum())
+               for g, dd in zip(v.reshape(-1, 128), d))
+    assert ties >= n                                   # the test really exercises ties
+    k = torch.from_numpy(v.copy()).bfloat16()
+    vt = torch.from_numpy(v).bfloat16()
+    oc, ost, gc, gst = _run_both(k, vt, orc.QUEST_INT, bits, [0], n)
+    assert ost == 0 and gst == 0
+    for name in ("v_meta", "v_codes", "k_meta", "k_codes"):
+        bad = np.argwhere(oc[name] != gc[name])
+        assert bad.size == 0, f"{name}: {len(bad)} mismatches, first {bad[:3].tolist()}"
