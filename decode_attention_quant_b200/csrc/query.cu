@@ -3,15 +3,16 @@
 // Keys are cached in the transformed basis x = T_k k (WUSH-KV: the key transform is
 // applied online after RoPE, ai4snews summary paragraph 5), so scores are kept
 // exact by mapping the query with the inverse-transpose: (T^{-T} q) . (T k) = q . k.
-// One CTA = one KV head and up to kBatchPerCta sequences; thread i owns output
-// channel i and keeps row i of T_k^{-T} in registers.
+// One CTA = one KV head of one sequence (its g query heads); thread i owns output
+// channel i, keeps row i of T_k^{-T} in registers and sums each product in four
+// interleaved chains, so the short launch is not one long dependent FMA chain.
 #include "wushkv_common.cuh"
 #include "wushkv_launch.h"
 
 namespace wushkv {
 namespace {
 
-constexpr int kBatchPerCta = 4;
+constexpr int kBatchPerCta = 1;
 
 template <bool BF16_IN>
 __global__ void __launch_bounds__(kHeadDim) transform_query_kernel(
@@ -39,17 +40,17 @@ __global__ void __launch_bounds__(kHeadDim) transform_query_kernel(
 #pragma unroll 1
   for (int r = 0; r < nb * g; ++r) {
     const float4* qr = reinterpret_cast<const float4*>(qs + r * kHeadDim);
-    float acc = 0.f;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
     for (int j = 0; j < kHeadDim / 4; ++j) {
       const float4 v = qr[j];
-      acc = fmaf(mr[4 * j], v.x, acc);
-      acc = fmaf(mr[4 * j + 1], v.y, acc);
-      acc = fmaf(mr[4 * j + 2], v.z, acc);
-      acc = fmaf(mr[4 * j + 3], v.w, acc);
+      a0 = fmaf(mr[4 * j], v.x, a0);
+      a1 = fmaf(mr[4 * j + 1], v.y, a1);
+      a2 = fmaf(mr[4 * j + 2], v.z, a2);
+      a3 = fmaf(mr[4 * j + 3], v.w, a3);
     }
     const int b = b0 + r / g, h = kv * g + r % g;
-    out[((size_t)b * hq + h) * kHeadDim + i] = acc;
+    out[((size_t)b * hq + h) * kHeadDim + i] = (a0 + a1) + (a2 + a3);
   }
 }
 
