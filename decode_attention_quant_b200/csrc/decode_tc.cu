@@ -5,8 +5,10 @@
 // both contractions run exactly as integer MMAs (tcgen05.mma kind::i8, int32
 // accumulate) and the fp16 meta is applied afterwards:
 //   scores  s_t = tau * (scale_t * sum_c q'_c code_tc + zero_t * sum_c q'_c)
-//           sum_c q'_c code_tc = (M / (2^22 - 1)) * sum_c qi_c code_tc, with q' rounded
-//           to 23-bit integers qi = l0 + 2^8 l1 + 2^16 l2 split into three int8 limbs;
+//           sum_c q'_c code_tc = (M / 2^30) * sum_c qi_c (f_c code_tc), where the key
+//           codes are widened by masking alone, so byte c holds f_c code_tc with a
+//           power of two f_c (see key_shift), and qi_c = rne(q'_c 2^30 / (M f_c)), M =
+//           max |q'|, is split into four int8 limbs qi = l0 + 2^8 l1 + 2^16 l2 + 2^24 l3;
 //   values  o_c = sum_t p_t (zero_t + scale_t code_tc)
 //               = (F / 65535) * sum_t pi_t code_tc + sum_t p_t zero_t,
 //           with p_t scale_t rounded to 16-bit integers pi = u0 + 2^8 u1 (per tile and
@@ -31,11 +33,12 @@
 // rewritten only after the event that ends its last read.  Two tokens per thread
 // halve the per-tile work (waits, maxima exchange, rescaling, accumulation) per
 // token.  Up to three CTAs run per SM (2-bit codes, g <= 8: two stages, ~73 KB shared
-// memory and 128 TMEM columns each); wider codes or groups run two.
-// 2- and 4-bit key codes are widened to bytes with two logic ops per 4 codes, which
-// permutes channels inside each 16 (8) channel block; the query limbs and the output
-// channels use the same permutation, so the contraction is unchanged.  Value codes
-// are widened by masking alone (see widen_row_scaled).
+// memory and 128 TMEM columns each); wider codes or groups run two (4-bit, g = 16: one).
+// 2- and 4-bit codes are widened to bytes by masking alone (one logic op per 4
+// codes), which permutes channels inside each 16 (8) channel block and leaves a
+// power-of-two factor on each channel; the query limbs and the output channels use
+// the same permutation, the query limbs divide the key factor out and the split
+// partial divides the value factor out, so both contractions are unchanged.
 #include <math_constants.h>
 
 #include <cmath>
@@ -55,7 +58,7 @@ constexpr int kTile = 2 * kHalf;        // tokens per pipeline step: two per tok
 constexpr int kThreads = 160;
 constexpr int kPartialStride = 132;     // m (log2 domain), l, pad, pad, o[128]
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kQScale = 4194303.0f;   // 2^22 - 1
+constexpr float kQScale = 1073741824.0f;  // 2^30: query integers up to 2^30 before the key factor
 constexpr uint32_t kBarTok = 1;         // named barrier of the four token warps
 constexpr int kSmemPerSm = 233472;      // bytes of shared memory per SM, 1 KB of it reserved per CTA
 
@@ -67,7 +70,7 @@ template <int BITS, int G>
 struct Cfg {
   static constexpr int kCode = 16 * BITS;                  // packed bytes per token row
   static constexpr int kStage = 2 * kTile * kCode;         // K then V codes of one tile
-  static constexpr int NK = round16(3 * G);                // score MMA N (3 limbs per head)
+  static constexpr int NK = round16(4 * G);                // score MMA N (4 limbs per head)
   static constexpr int NV = round16(2 * G);                // value MMA N (2 limbs per head)
   static constexpr int kColAk = 0;                         // 2 halves x 32 columns (u8 x 128 channels)
   static constexpr int kColS = 64;                         // 2 halves x NK
@@ -79,7 +82,7 @@ struct Cfg {
   static constexpr int kFixed = 2 * kHalf * 128 + 2 * NV * 128 + NK * 128 + 2048 + 1024;
   // as many resident CTAs per SM (up to 3) as leave room for a double-buffered ring
   static constexpr int ring(int ctas) { return (kSmemPerSm / ctas - 1024 - kFixed) / kStage; }
-  static constexpr int kCtas = ring(3) >= 2 ? 3 : 2;
+  static constexpr int kCtas = ring(3) >= 2 ? 3 : ring(2) >= 2 ? 2 : 1;
   static constexpr int kSmemPerCta = kSmemPerSm / kCtas - 1024;
   static constexpr int kStages = cmin(4, ring(kCtas));
   static constexpr int kOffStage = 0;
@@ -189,6 +192,15 @@ __device__ __forceinline__ void widen_row_scaled(const uint8_t* row, uint32_t (&
   }
 }
 
+// log2 of the factor the masked widening leaves on channel c (2-bit: 4^(c & 3);
+// 4-bit: 16^(c & 1); 3-bit: none), for key and value codes alike
+template <int BITS>
+__device__ __forceinline__ int key_shift(int c) {
+  if (BITS == 2) return 2 * (c & 3);
+  if (BITS == 4) return 4 * (c & 1);
+  return 0;
+}
+
 template <int BITS>
 __device__ __forceinline__ float value_scale_of(int p) {
   if (BITS == 2) return (float)(1 << (2 * ((p >> 2) & 3)));
@@ -282,22 +294,26 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       const float qv = a.q[((size_t)b * a.hq + kv * G + h) * kHeadDim + c];
       const float4 m4 = ms->red[0][h];
       const float mx = fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w));
-      const float inv = mx > 0.f ? kQScale / mx : 0.f;
-      const int qi = __float2int_rn(qv * inv);              // |qi| <= 2^22 - 1
+      // the key byte of channel c carries 2^key_shift(c): divide it out of q' exactly
+      const float inv = mx > 0.f ? kQScale / mx * __int_as_float((127 - key_shift<BITS>(c)) << 23) : 0.f;
+      const int qi = __float2int_rn(qv * inv);              // |qi| <= 2^30
       const int l0 = (int)(int8_t)(qi & 0xff);
       const int r1 = (qi - l0) >> 8;
       const int l1 = (int)(int8_t)(r1 & 0xff);
-      const int l2 = (r1 - l1) >> 8;                        // |l2| <= 64
+      const int r2 = (r1 - l1) >> 8;
+      const int l2 = (int)(int8_t)(r2 & 0xff);
+      const int l3 = (r2 - l2) >> 8;                        // |l3| <= 64
       bk[kmajor_off(h, p)] = (uint8_t)l0;
       bk[kmajor_off(G + h, p)] = (uint8_t)l1;
       bk[kmajor_off(2 * G + h, p)] = (uint8_t)l2;
+      bk[kmajor_off(3 * G + h, p)] = (uint8_t)l3;
       if (p == 0) {
         const float4 s4 = ms->red[1][h];
         ms->c1[h] = (mx > 0.f ? mx / kQScale : 0.f) * a.scale_log2;
         ms->c2[h] = ((s4.x + s4.y) + (s4.z + s4.w)) * a.scale_log2;
       }
     }
-    for (int nrow = 3 * G; nrow < C::NK; ++nrow) bk[kmajor_off(nrow, p)] = 0;
+    for (int nrow = 4 * G; nrow < C::NK; ++nrow) bk[kmajor_off(nrow, p)] = 0;
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -402,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint32_t wv[32];
-          widen_row<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, wv);
+          widen_row_scaled<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, wv);
           tmem_st32(tmem + lanes + C::kColAk + 32 * j, wv);
         }
         tmem_st_wait();
@@ -458,8 +474,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const int si = (int)d[h] + (int)d[G + h] * 256 + (int)d[2 * G + h] * 65536;
-          const float dot = fmaf(ks[j], (float)si * c1[h], kz[j] * c2[h]);
+          // |limb sum| <= 128 * 240 * 128, so two limbs combine exactly in int32
+          const int lo = (int)d[h] + (int)d[G + h] * 256;
+          const int hi = (int)d[2 * G + h] + (int)d[3 * G + h] * 256;
+          const float si = fmaf((float)hi, 65536.0f, (float)lo);
+          const float dot = fmaf(ks[j], si * c1[h], kz[j] * c2[h]);
           s2[j][h] = valid[j] ? dot : -CUDART_INF_F;
         }
       }
@@ -655,9 +674,10 @@ cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaS
 // Resident decode CTAs per SM for a cache's bit width and group size (Cfg::kCtas).
 int ctas_per_sm(int bits, int g) {
   static_assert(Cfg<2, 8>::kCtas == 3 && Cfg<2, 16>::kCtas == 2 && Cfg<3, 1>::kCtas == 2 &&
-                    Cfg<4, 1>::kCtas == 2 && Cfg<4, 16>::kCtas == 2,
+                    Cfg<3, 16>::kCtas == 2 && Cfg<4, 8>::kCtas == 2 && Cfg<4, 16>::kCtas == 1,
                 "keep ctas_per_sm in step with Cfg");
-  return (bits == 2 && g <= 8) ? 3 : 2;
+  if (bits == 2 && g <= 8) return 3;
+  return (bits == 4 && g >= 16) ? 1 : 2;
 }
 
 }  // namespace
