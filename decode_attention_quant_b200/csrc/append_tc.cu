@@ -206,10 +206,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     bars->abort = 0;
     fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
+    // the first fill of both rings goes out now, so it overlaps the transform split
     tma_prefetch(&kmap);
     tma_prefetch(&vmap);
+    for (int li = 0; li < n_loc && li < kStages; ++li) {
+      const int tile = j0 + li * a.ctas_per_head;
+      mbar_arrive_expect_tx(&bars->full_k[li], kTileBytes);
+      tma_load_3d(kst + li * kTileBytes, &kmap, &bars->full_k[li], 0, h, tile * kRowsPerTile);
+      tma_load_3d(kst + li * kTileBytes + kBoxBytes, &kmap, &bars->full_k[li], 64, h, tile * kRowsPerTile);
+      mbar_arrive_expect_tx(&bars->full_v[li], kTileBytes);
+      tma_load_3d(vst + li * kTileBytes, &vmap, &bars->full_v[li], 0, h, tile * kRowsPerTile);
+      tma_load_3d(vst + li * kTileBytes + kBoxBytes, &vmap, &bars->full_v[li], 64, h, tile * kRowsPerTile);
+    }
   }
   if (HAS_T) {
     if (warp == 1) {
@@ -228,8 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      int issued_k = 0, issued_v = 0;
-      for (int li = 0; li < n_loc; ++li) {
+      const int first = n_loc < kStages ? n_loc : kStages;   // issued before the split
+      int issued_k = first, issued_v = first;
+      for (int li = first; li < n_loc; ++li) {
         const int tile = j0 + li * a.ctas_per_head;
         const int s = li % kStages;
         const uint32_t ph = (li / kStages) & 1;

@@ -619,23 +619,42 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
   }
 }
 
-// out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s   (log2-domain partials)
+// out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s   (log2-domain partials).
+// One pass over the splits in batches of eight whose loads are all in flight at once,
+// rescaling the running sums whenever a batch raises the maximum.
+constexpr int kCombineBatch = 8;
 __global__ void __launch_bounds__(kHeadDim) combine_log2_kernel(const float* __restrict__ ws, int num_splits,
                                                                float* __restrict__ out) {
   const size_t bh = blockIdx.x;
   const int c = threadIdx.x;
   const float* p = ws + bh * num_splits * kPartialStride;
-  float mx = -CUDART_INF_F;
-  for (int s = 0; s < num_splits; ++s) mx = fmaxf(mx, p[s * kPartialStride]);
-  float l = 0.f, o = 0.f;
-  if (mx > -CUDART_INF_F) {
-    for (int s = 0; s < num_splits; ++s) {
-      const float ms = p[s * kPartialStride];
-      if (ms == -CUDART_INF_F) continue;
-      const float w = exp2f(ms - mx);
-      l = fmaf(w, p[s * kPartialStride + 1], l);
-      o = fmaf(w, p[s * kPartialStride + 4 + c], o);
+  float mx = -CUDART_INF_F, l = 0.f, o = 0.f;
+  for (int s0 = 0; s0 < num_splits; s0 += kCombineBatch) {
+    float mv[kCombineBatch], lv[kCombineBatch], ov[kCombineBatch];
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) {
+      const bool in = s0 + k < num_splits;
+      const float* ps = p + (size_t)(s0 + k) * kPartialStride;
+      mv[k] = in ? __ldg(ps) : -CUDART_INF_F;
+      lv[k] = in ? __ldg(ps + 1) : 0.f;
+      ov[k] = in ? __ldg(ps + 4 + c) : 0.f;
     }
+    float bm = mv[0];
+#pragma unroll
+    for (int k = 1; k < kCombineBatch; ++k) bm = fmaxf(bm, mv[k]);
+    const float nm = fmaxf(mx, bm);
+    if (nm == -CUDART_INF_F) continue;            // nothing seen yet
+    const float sc = exp2f(mx - nm);              // 0 while mx is still -inf
+    l *= sc;
+    o *= sc;
+#pragma unroll
+    for (int k = 0; k < kCombineBatch; ++k) {
+      if (mv[k] == -CUDART_INF_F) continue;       // empty split (or past the end)
+      const float w = exp2f(mv[k] - nm);
+      l = fmaf(w, lv[k], l);
+      o = fmaf(w, ov[k], o);
+    }
+    mx = nm;
   }
   out[bh * kHeadDim + c] = l > 0.f ? o / l : 0.f;
 }
