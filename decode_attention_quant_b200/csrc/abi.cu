@@ -15,6 +15,9 @@ cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, 
 cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new, const void* v_new,
                                         int in_dtype, int n_new, const int32_t* start_pos,
                                         const float* Tk, int32_t* status, cudaStream_t stream);
+cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
+                                         const int32_t* start_pos, const float* Tk, int32_t* status,
+                                         cudaStream_t stream);
 }
 
 namespace {
@@ -79,14 +82,19 @@ int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const v
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(start_pos, 4)) return WUSHKV_ERR_MISALIGNED;
   if (Tk != nullptr && !aligned(Tk, 16)) return WUSHKV_ERR_MISALIGNED;
   if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
-  // bf16 rows (the serving path) go through TMA + tcgen05; fp32 rows (exact pre-transformed
-  // values, used to test the quantizer alone) through the per-row kernel.  Both share the
-  // quantizer code.
+  // bf16 rows (the serving path) go through TMA + tcgen05, except a decode step's few
+  // rows, which a latency-oriented kernel (one warp per group) takes; fp32 rows (exact
+  // pre-transformed values, used to test the quantizer alone) go through the per-row
+  // kernel.  All decide every code exactly for the fp32 value they quantize.
+  constexpr int64_t kSmallAppendRows = 64;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = in_dtype == WUSHKV_BF16
-                      ? wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st)
-                      : wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos, Tk,
-                                                            status, st);
+  cudaError_t e;
+  if (in_dtype == WUSHKV_BF16 && (int64_t)cache->batch * n_new <= kSmallAppendRows)
+    e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
+  else if (in_dtype == WUSHKV_BF16)
+    e = wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
+  else
+    e = wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos, Tk, status, st);
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 

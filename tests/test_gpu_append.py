@@ -229,3 +229,29 @@ def test_bf16_values_on_thresholds_bitexact(bits):
     for name in ("v_meta", "v_codes", "k_meta", "k_codes"):
         bad = np.argwhere(oc[name] != gc[name])
         assert bad.size == 0, f"{name}: {len(bad)} mismatches, first {bad[:3].tolist()}"
+
+
+@pytest.mark.parametrize("kind,bits", CASES)
+@pytest.mark.parametrize("bsz,n", [(16, 1), (4, 16)])
+def test_small_append_end_to_end(kind, bits, bsz, n):
+    """Decode-step sized appends (<= 64 rows) take the one-warp-per-group kernel: same
+    bar as the bulk path (value codes/meta bit-exact; key rules as above)."""
+    w = QWEN8B_DECODE
+    hkv, cap = 2, 48
+    start = [(7 * b) % 30 for b in range(bsz)]
+    tk = torch.from_numpy(gen.transforms(w)[0][:hkv].copy())
+    k = gen.keys(w, 0, bsz, start, n)[:, :, :hkv].contiguous()
+    v = gen.values(w, 0, bsz, start, n)[:, :, :hkv].contiguous()
+    _e2e_check(k, v, tk, kind, bits, start, cap)
+
+
+def test_small_append_capacity_and_status():
+    """Rows past the capacity are skipped with status bit 1 on the small path too."""
+    w = QWEN8B_DECODE
+    k = gen.keys(w, 0, 3, [0, 0, 0], 1)[:, :, :1].contiguous()
+    v = gen.values(w, 0, 3, [0, 0, 0], 1)[:, :, :1].contiguous()
+    tk = torch.from_numpy(gen.transforms(w)[0][:1].copy())
+    oc, ost, gc, gst = _run_both(k, v, 1, 2, [5, 9, 2], 9, tk=tk)       # sequence 1 writes position 9 = cap
+    assert ost & orc.STATUS_CAPACITY and gst & dq.STATUS_CAPACITY
+    np.testing.assert_array_equal(oc["v_codes"], gc["v_codes"])
+    np.testing.assert_array_equal(oc["v_meta"], gc["v_meta"])
