@@ -141,10 +141,8 @@ __device__ __forceinline__ void load_row(const uint8_t* row, uint32_t (&w)[4 * B
 }
 
 template <int BITS>
-__device__ __forceinline__ void widen_row(const uint8_t* row, uint32_t (&u)[32]) {
+__device__ __forceinline__ void widen_words(const uint32_t (&w)[4 * BITS], uint32_t (&u)[32]) {
   constexpr int kWords = 4 * BITS;
-  uint32_t w[kWords];
-  load_row<BITS>(row, w);
   if (BITS == 2) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -167,18 +165,16 @@ __device__ __forceinline__ void widen_row(const uint8_t* row, uint32_t (&u)[32])
   }
 }
 
-// Value codes are widened by masking alone: byte p then holds code * value_scale_of(p)
-// (2-bit: 4^((p >> 2) & 3); 4-bit: 16^((p >> 2) & 1); 3-bit: 1).  Position p is an
-// output channel of the value MMA, so the power of two is divided out exactly once,
-// from the split partial.  Largest int32 sum per tile: 65535 * 240 * 128 < 2^31.
+// Codes widened by masking alone: byte p then holds code * 2^key_shift(channel_of(p))
+// (2-bit: 4^((p >> 2) & 3); 4-bit: 16^((p >> 2) & 1); 3-bit: the shifted form above,
+// factor 1).  Bytes stay <= 240, so every MMA limb column fits int32 (score: 128 * 240 *
+// 128 per channel sum; value: 255 * 240 * 256 per tile).
 template <int BITS>
-__device__ __forceinline__ void widen_row_scaled(const uint8_t* row, uint32_t (&u)[32]) {
+__device__ __forceinline__ void widen_words_scaled(const uint32_t (&w)[4 * BITS], uint32_t (&u)[32]) {
   if (BITS == 3) {
-    widen_row<BITS>(row, u);
+    widen_words<BITS>(w, u);
     return;
   }
-  uint32_t w[4 * BITS];
-  load_row<BITS>(row, w);
   if (BITS == 2) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)
@@ -415,10 +411,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
         }
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / S) & 1, abort));
       if (ok) {
+        uint32_t w[2][4 * BITS];                // both rows' loads in flight before widening
+#pragma unroll
+        for (int j = 0; j < 2; ++j) load_row<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, w[j]);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint32_t wv[32];
-          widen_row_scaled<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, wv);
+          widen_words_scaled<BITS>(w[j], wv);
           tmem_st32(tmem + lanes + C::kColAk + 32 * j, wv);
         }
         tmem_st_wait();
@@ -432,10 +431,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
     auto widen_v = [&](int i) {
       const int s = i % S;
       if (ok) {
+        uint32_t w[2][4 * BITS];                // both rows' loads in flight before the stores
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          load_row<BITS>(stage + s * C::kStage + kTile * C::kCode + (r + kHalf * j) * C::kCode, w[j]);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint32_t wv[32];
-          widen_row_scaled<BITS>(stage + s * C::kStage + kTile * C::kCode + (r + kHalf * j) * C::kCode, wv);
+          widen_words_scaled<BITS>(w[j], wv);
           uint8_t* arow = av + j * kHalf * 128 + r * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
@@ -465,13 +468,26 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->kdone, u, abort));
       tc_fence_after();
       float s2[2][G];
+      constexpr bool kOneWait = 2 * C::NK <= 32;   // both halves' limbs in flight together
+      uint32_t dd[kOneWait ? 2 : 1][C::NK];
+      if (kOneWait) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int c0 = 0; c0 < C::NK; c0 += 16)
+            tmem_ld16(tmem + lanes + C::kColS + j * C::NK + c0,
+                      *reinterpret_cast<uint32_t(*)[16]>(dd[kOneWait ? j : 0] + c0));
+        tmem_ld_wait();
+      }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        uint32_t d[C::NK];
+        uint32_t* d = dd[kOneWait ? j : 0];
+        if (!kOneWait) {
 #pragma unroll
-        for (int c0 = 0; c0 < C::NK; c0 += 16)
-          tmem_ld16(tmem + lanes + C::kColS + j * C::NK + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
-        tmem_ld_wait();
+          for (int c0 = 0; c0 < C::NK; c0 += 16)
+            tmem_ld16(tmem + lanes + C::kColS + j * C::NK + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
+          tmem_ld_wait();
+        }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           // |limb sum| <= 128 * 240 * 128, so two limbs combine exactly in int32
@@ -570,8 +586,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const int di = (int)d[h] + (int)d[G + h] * 256;
-          o[h] = fmaf(o[h], corr[h], fs[h] * (float)di);
+          // each limb column is <= 255 * 240 * 256 (exact int32); their combination can
+          // pass 2^31 when attention is flat over the tile, so it is formed in fp32
+          const float di = fmaf((float)(int)d[G + h], 256.0f, (float)(int)d[h]);
+          o[h] = fmaf(o[h], corr[h], fs[h] * di);
         }
       }
       tc_fence_before();

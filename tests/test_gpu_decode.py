@@ -120,3 +120,31 @@ def test_decode_full_size_sampled(kind, bits, batch, hq, hkv, ctx):
         ref = orc.decode_attention_pair(kc, km, vc, vm, qn[b, kv * gsz:(kv + 1) * gsz], TAU, kind, bits)
         ma, rl = gu.attention_errors(out[b, kv * gsz:(kv + 1) * gsz], ref)
         assert ma <= MAX_ABS and rl <= REL_L2, (b, kv, ma, rl)
+
+
+@pytest.mark.parametrize("kind,bits", [(1, 2), (0, 2), (0, 3), (1, 4)])
+def test_flat_attention_over_maximal_value_codes(kind, bits):
+    """Equal scores over whole tiles and every value code at its maximum: the largest
+    value sums a tile can produce (each limb column near 255 x 240 x 256), so any int32
+    overflow in combining them would show.  The output is the dequantized top code."""
+    bsz, hkv, hq, ctx = 2, 2, 8, 1024
+    c = gen.random_cache(bsz, hkv, ctx, kind, bits, seed=7, device="cpu")
+    c["k_codes"][:] = c["k_codes"][:, :, :1].clone()          # one key row repeated: equal scores
+    c["k_meta"][:] = c["k_meta"][:, :, :1].clone()
+    c["v_codes"][:] = 0xFF                                     # every value code = 2^b - 1
+    c["v_meta"][:] = c["v_meta"][:, :, :1].clone()             # equal value scales: e * scale at the cap
+    cache = dq.PackedCache(bsz, hkv, ctx, kind, bits, tensors={k: v.cuda() for k, v in c.items()})
+    q = torch.randn(bsz, hq, 128, generator=torch.Generator().manual_seed(4)) * 2.0
+    ctx_t = torch.full((bsz,), ctx, dtype=torch.int32, device="cuda")
+    for ns in (0, 1):                                          # automatic split count, and one split
+        out = dq.decode_attention(cache, q.cuda(), ctx_t, TAU, num_splits=ns).cpu().numpy()
+        gsz = hq // hkv
+        for b in range(bsz):
+            for kv in range(hkv):
+                km = c["k_meta"][b, kv].numpy().view(np.uint16)
+                vm = c["v_meta"][b, kv].numpy().view(np.uint16)
+                ref = orc.decode_attention_pair(c["k_codes"][b, kv].numpy(), km, c["v_codes"][b, kv].numpy(), vm,
+                                                q[b, kv * gsz:(kv + 1) * gsz].numpy().astype(np.float64), TAU,
+                                                kind, bits)
+                ma, rl = gu.attention_errors(out[b, kv * gsz:(kv + 1) * gsz], ref)
+                assert ma <= MAX_ABS and rl <= REL_L2, (ns, b, kv, ma, rl)
