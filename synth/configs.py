@@ -71,23 +71,23 @@ class Workload:
         return self.num_q_heads // self.num_kv_heads
 
 
-# configs[0]: tiny single layer; history = the 256 prompt tokens, QuEST 2-bit
+# Tiny single layer; history = the 256 prompt tokens, QuEST 2-bit
 TINY = Workload("tiny_b1_h4kv1_t256_quest2", batch=1, num_q_heads=4, num_kv_heads=1,
                 ctx=256, quant=quest(2), history=0, append_tokens=256, seed=1000)
-# configs[1]: Qwen3-8B-shaped decode layer, percentile-affine 2-bit
+# Qwen3-8B-shaped decode layer, percentile-affine 2-bit
 QWEN8B_DECODE = Workload("qwen3_8b_b16_ctx32768_affine2", batch=16, num_q_heads=32,
                          num_kv_heads=8, ctx=32768, quant=affine(2), history=32767,
                          append_tokens=1, value_heavy=(3, 17), seed=2000)
-# configs[2]: QuEST sweep on the Qwen3-8B shapes: 2048-token chunk appended after 30720
+# QuEST bit-width sweep on the Qwen3-8B shapes: 2048-token chunk appended after 30720
 def QWEN8B_SWEEP(bits: int) -> Workload:
     return Workload(f"qwen3_8b_b16_chunk2048_quest{bits}", batch=16, num_q_heads=32,
                     num_kv_heads=8, ctx=32768, quant=quest(bits), history=30720,
                     append_tokens=2048, value_heavy=(3, 17), seed=3000 + bits)
-# configs[3]: long-context decode, split-K
+# Long-context decode, split-K
 QWEN8B_LONG = Workload("qwen3_8b_b4_ctx131072_affine2", batch=4, num_q_heads=32,
                        num_kv_heads=8, ctx=131072, quant=affine(2), history=131071,
                        append_tokens=1, value_heavy=(3, 17), seed=4000)
-# configs[4]: Qwen3-32B-shaped 64-layer stack, 16-token chunk per layer
+# Qwen3-32B-shaped 64-layer stack, 16-token chunk per layer
 QWEN32B_STACK = Workload("qwen3_32b_64l_b32_ctx8192_quest2", batch=32, num_q_heads=64,
                          num_kv_heads=8, ctx=8192, quant=quest(2), layers=64,
                          history=8176, append_tokens=16, value_heavy=(3, 17), seed=5000)
