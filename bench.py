@@ -246,31 +246,52 @@ def run_ours(args, rank, world, local):
             step()
         torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # external: when captured into a graph, the records stay timestamped event nodes
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True, external=True)
+    t1 = torch.cuda.Event(enable_timing=True, external=True)
+
+    def timed_steps(s):
+        t0.record(s)
+        for i in range(args.steps):
+            ev[i][0].record(s)
+            dq.quantize_append(cache, k_new, v_new, start, tk, status)
+            ev[i][1].record(s)
+            dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
+            ev[i][2].record(s)
+            dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+            ev[i][3].record(s)
+        t1.record(s)
+
+    # The K timed steps are captured once into a CUDA graph (the library's calls allocate
+    # and synchronise nothing) and replayed once, so the host's per-call Python overhead
+    # cannot leave the device idle between launches; eager launches if capture fails.
+    graph = None
+    if not args.eager:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                timed_steps(torch.cuda.current_stream())
+        except Exception as exc:  # noqa: BLE001 - report and time the eager loop instead
+            print(f"graph capture failed ({exc}); timing eager launches", file=sys.stderr)
+            graph = None
     barrier(world)
     torch.cuda.synchronize()
-    if True:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.nvtx.range_push("timed_steps")       # lets a profiler select these launches
-        t0.record(stream)
-        for i in range(args.steps):
-            ev[i][0].record(stream)
-            dq.quantize_append(cache, k_new, v_new, start, tk, status)
-            ev[i][1].record(stream)
-            dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
-            ev[i][2].record(stream)
-            dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
-            ev[i][3].record(stream)
-        t1.record(stream)
-        torch.cuda.nvtx.range_pop()
-        torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed_steps")           # lets a profiler select these launches
+    if graph is not None:
+        graph.replay()
+    else:
+        timed_steps(stream)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
     timed_to = time.time()
     clk.__exit__(None, None, None)
     barrier(world)
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
     ms_step = ms_total / args.steps
     dec_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps))
+    breakdown = {name: round(statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)), 5)
+                 for j, name in enumerate(("append_ms", "query_map_ms", "decode_ms"))}
     step_bytes = decode_bytes(w, [w.ctx] * w.batch) + append_bytes(w, 1) + query_bytes(w)
     value = world * step_bytes / (ms_step * 1e-3) / 1e9
     peak, peak_kind = _peaks()
@@ -318,8 +339,10 @@ def run_ours(args, rank, world, local):
         "config": {"workload": f"{w.name}: 1-token append + query map + split-K decode per step",
                    "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
                    "head_dim": 128, "ctx": w.ctx, "quantizer": "percentile-affine 2-bit ranks 2/125",
-                   "l2": "inputs larger than L2 (packed cache 302 MB > 126 MB L2)", "parallelism": f"replicas x{world}"},
+                   "l2": "inputs larger than L2 (packed cache 302 MB > 126 MB L2)", "parallelism": f"replicas x{world}",
+                   "launch": "one CUDA graph of the timed steps" if graph is not None else "eager launches"},
         "step_bytes": step_bytes,
+        "step_breakdown": breakdown,
         "roofline": {"bound": "hbm", "kernel": "decode call (split-K decode_tc_kernel + combine)",
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": profiled_decode_traffic(),
@@ -451,6 +474,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a captured graph")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
