@@ -17,8 +17,8 @@
 // log2 domain across 128-token tiles.
 //
 // One CTA = one (sequence, KV head, split); tiles of 256 tokens, five warps:
-//   warp 0      one thread: bulk copies of each tile's packed K and V codes into a
-//               ring of stages, and every MMA, each issued when the mbarrier of the
+//   warp 0      one thread: TMA copies of each tile's packed K and V codes into a
+//               ring of stages (swizzled so the row reads are bank-conflict free), and every MMA, each issued when the mbarrier of the
 //               event it needs completes (key codes widened; probabilities written).
 //   warps 1-4   token warps.  Thread = tokens r and 128 + r of the tile (lane r of
 //               the two M = 128 score MMAs) while widening codes to u8 (K codes into
@@ -130,12 +130,23 @@ __device__ __forceinline__ int channel_of(int p) {
   return p;
 }
 
-// Packed row (16*BITS bytes at `row`) -> 32 words of four u8 codes (K order as above).
+// TMA swizzle of a stage's code rows: 2-bit rows (32 B) use the 32-byte pattern, 4-bit
+// rows (64 B) the 64-byte one (16-byte chunk index XOR address bits 7.. of the row), so
+// the 16-byte reads of eight consecutive rows hit distinct banks; 3-bit rows (48 B) are
+// conflict-free unswizzled.
 template <int BITS>
-__device__ __forceinline__ void load_row(const uint8_t* row, uint32_t (&w)[4 * BITS]) {
+__host__ __device__ constexpr int code_swizzle(int row) {
+  return BITS == 2 ? ((row >> 2) & 1) : BITS == 4 ? ((row >> 1) & 3) : 0;
+}
+
+// Packed row `row` of a stage's code tile (16*BITS bytes per row) -> 4*BITS words.
+template <int BITS>
+__device__ __forceinline__ void load_row(const uint8_t* tile, int row, uint32_t (&w)[4 * BITS]) {
+  const uint8_t* p = tile + row * (16 * BITS);
+  const int sw = code_swizzle<BITS>(row);
 #pragma unroll
   for (int q = 0; q < BITS; ++q) {
-    const uint4 v = *reinterpret_cast<const uint4*>(row + 16 * q);
+    const uint4 v = *reinterpret_cast<const uint4*>(p + 16 * (q ^ sw));
     w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
   }
 }
@@ -227,7 +238,8 @@ __device__ __forceinline__ int kmajor_off(int n, int k) {
 }
 
 template <int BITS, int KIND, int G>
-__global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kernel(DecArgs a) {
+__global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, DecArgs a) {
   using C = Cfg<BITS, G>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -327,15 +339,17 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       constexpr uint32_t kIdK = idesc(kFmtS32, kFmtU8, kFmtS8, 0, 0, 128, C::NK);
       constexpr uint32_t kIdV = idesc(kFmtS32, kFmtU8, kFmtU8, 1, 1, 128, C::NV);
       const uint32_t bk_addr = smem_u32(bk), bv_addr = smem_u32(bv), av_addr = smem_u32(av);
+      tma_prefetch(&kmap);
+      tma_prefetch(&vmap);
       int issued = 0;
+      // a tile's K and V code rows, one 3-D box each ([pair][token][byte], swizzled);
+      // rows past the capacity arrive as zeros, rows past the context are never used
       auto load = [&](int i) {
         const int s = i % S;
         const int t0 = (tile0 + i) * kTile;
-        const uint32_t bytes = (uint32_t)min(kTile, L - t0) * C::kCode;
-        mbar_arrive_expect_tx(&ms->full[s], 2 * bytes);
-        const size_t off = (pair * a.capacity + t0) * C::kCode;
-        bulk_load(stage + s * C::kStage, a.k_codes + off, bytes, &ms->full[s]);
-        bulk_load(stage + s * C::kStage + kTile * C::kCode, a.v_codes + off, bytes, &ms->full[s]);
+        mbar_arrive_expect_tx(&ms->full[s], 2 * kTile * C::kCode);
+        tma_load_3d(stage + s * C::kStage, &kmap, &ms->full[s], 0, t0, (int)pair);
+        tma_load_3d(stage + s * C::kStage + kTile * C::kCode, &vmap, &ms->full[s], 0, t0, (int)pair);
         ++issued;
       };
       auto score_mma = [&]() {
@@ -413,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       if (ok) {
         uint32_t w[2][4 * BITS];                // both rows' loads in flight before widening
 #pragma unroll
-        for (int j = 0; j < 2; ++j) load_row<BITS>(stage + s * C::kStage + (r + kHalf * j) * C::kCode, w[j]);
+        for (int j = 0; j < 2; ++j) load_row<BITS>(stage + s * C::kStage, r + kHalf * j, w[j]);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint32_t wv[32];
@@ -433,8 +447,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas) decode_tc_kerne
       if (ok) {
         uint32_t w[2][4 * BITS];                // both rows' loads in flight before the stores
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-          load_row<BITS>(stage + s * C::kStage + kTile * C::kCode + (r + kHalf * j) * C::kCode, w[j]);
+        for (int j = 0; j < 2; ++j) load_row<BITS>(stage + s * C::kStage + kTile * C::kCode, r + kHalf * j, w[j]);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           uint32_t wv[32];
@@ -677,14 +690,30 @@ __global__ void __launch_bounds__(kHeadDim) combine_log2_kernel(const float* __r
   out[bh * kHeadDim + c] = l > 0.f ? o / l : 0.f;
 }
 
+// Tensor map over one side's codes: [pairs][capacity][16*BITS bytes], boxes of a tile's
+// 256 rows, swizzled as code_swizzle describes.
+template <int BITS>
+bool code_map(CUtensorMap* m, const uint8_t* base, int capacity, int pairs) {
+  const uint64_t dims[3] = {(uint64_t)(16 * BITS), (uint64_t)capacity, (uint64_t)pairs};
+  const uint64_t strides[2] = {(uint64_t)(16 * BITS), (uint64_t)capacity * (16 * BITS)};
+  const uint32_t box[3] = {(uint32_t)(16 * BITS), (uint32_t)kTile, 1};
+  const CUtensorMapSwizzle sw = BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                : BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, sw);
+}
+
 template <int BITS, int KIND, int G>
 cudaError_t launch_g(const DecArgs& a, int batch, float* out, cudaStream_t stream) {
   using C = Cfg<BITS, G>;
   auto kern = decode_tc_kernel<BITS, KIND, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
+  CUtensorMap km, vm;
+  if (!code_map<BITS>(&km, a.k_codes, a.capacity, batch * a.hkv) || !code_map<BITS>(&vm, a.v_codes, a.capacity, batch * a.hkv))
+    return cudaErrorInvalidValue;
   dim3 grid(a.num_splits, a.hkv, batch);
-  kern<<<grid, kThreads, C::kSmem, stream>>>(a);
+  kern<<<grid, kThreads, C::kSmem, stream>>>(km, vm, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   combine_log2_kernel<<<batch * a.hq, kHeadDim, 0, stream>>>(a.ws, a.num_splits, out);
