@@ -251,30 +251,42 @@ def run_ours(args, rank, world, local):
     t0 = torch.cuda.Event(enable_timing=True, external=True)
     t1 = torch.cuda.Event(enable_timing=True, external=True)
 
+    def steps(s, per_launch):
+        for i in range(args.steps):
+            if per_launch:
+                ev[i][0].record(s)
+            dq.quantize_append(cache, k_new, v_new, start, tk, status)
+            if per_launch:
+                ev[i][1].record(s)
+            dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
+            if per_launch:
+                ev[i][2].record(s)
+            dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+            if per_launch:
+                ev[i][3].record(s)
+
     def timed_steps(s):
         t0.record(s)
-        for i in range(args.steps):
-            ev[i][0].record(s)
-            dq.quantize_append(cache, k_new, v_new, start, tk, status)
-            ev[i][1].record(s)
-            dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
-            ev[i][2].record(s)
-            dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
-            ev[i][3].record(s)
+        steps(s, False)
         t1.record(s)
 
     # The K timed steps are captured once into a CUDA graph (the library's calls allocate
     # and synchronise nothing) and replayed once, so the host's per-call Python overhead
-    # cannot leave the device idle between launches; eager launches if capture fails.
-    graph = None
+    # cannot leave the device idle between launches; eager launches if capture fails.  A
+    # second graph of the same steps with an event around every launch gives the per-call
+    # times (decode roofline, step breakdown) without adding event records to the timed one.
+    graph = graph_ev = None
     if not args.eager:
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 timed_steps(torch.cuda.current_stream())
+            graph_ev = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_ev):
+                steps(torch.cuda.current_stream(), True)
         except Exception as exc:  # noqa: BLE001 - report and time the eager loop instead
             print(f"graph capture failed ({exc}); timing eager launches", file=sys.stderr)
-            graph = None
+            graph = graph_ev = None
     barrier(world)
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_push("timed_steps")           # lets a profiler select these launches
@@ -286,8 +298,13 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     timed_to = time.time()
     clk.__exit__(None, None, None)
-    barrier(world)
     ms_total = max_over_ranks(t0.elapsed_time(t1), world)
+    if graph_ev is not None:                            # per-call times, outside the timed region
+        graph_ev.replay()
+    else:
+        steps(stream, True)
+    torch.cuda.synchronize()
+    barrier(world)
     ms_step = ms_total / args.steps
     dec_ms = statistics.mean(ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps))
     breakdown = {name: round(statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)), 5)
