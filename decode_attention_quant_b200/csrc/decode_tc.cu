@@ -32,7 +32,7 @@
 // [score MMAs(i+1)]; accumulate(i); widen V(i+1).  Every buffer is single: each is
 // rewritten only after the event that ends its last read.  Two tokens per thread
 // halve the per-tile work (waits, maxima exchange, rescaling, accumulation) per
-// token.  Up to three CTAs run per SM (2-bit codes, g <= 8: two stages, ~73 KB shared
+// token.  Up to three CTAs run per SM (2-bit codes, g <= 4: two stages, ~73 KB shared
 // memory and 128 TMEM columns each); wider codes or groups run two (4-bit, g = 16: one).
 // 2- and 4-bit codes are widened to bytes by masking alone (one logic op per 4
 // codes), which permutes channels inside each 16 (8) channel block and leaves a
@@ -82,7 +82,8 @@ struct Cfg {
   static constexpr int kFixed = 2 * kHalf * 128 + 2 * NV * 128 + NK * 128 + 2048 + 1024;
   // as many resident CTAs per SM (up to 3) as leave room for a double-buffered ring
   static constexpr int ring(int ctas) { return (kSmemPerSm / ctas - 1024 - kFixed) / kStage; }
-  static constexpr int kCtas = ring(3) >= 2 ? 3 : ring(2) >= 2 ? 2 : 1;
+  // (g = 8 would need more than the 128 registers three CTAs leave a thread: two)
+  static constexpr int kCtas = (ring(3) >= 2 && G <= 4) ? 3 : ring(2) >= 2 ? 2 : 1;
   static constexpr int kSmemPerCta = kSmemPerSm / kCtas - 1024;
   static constexpr int kStages = cmin(4, ring(kCtas));
   static constexpr int kOffStage = 0;
@@ -739,10 +740,10 @@ cudaError_t launch_bits(const DecArgs& a, int kind, int batch, float* out, cudaS
 
 // Resident decode CTAs per SM for a cache's bit width and group size (Cfg::kCtas).
 int ctas_per_sm(int bits, int g) {
-  static_assert(Cfg<2, 8>::kCtas == 3 && Cfg<2, 16>::kCtas == 2 && Cfg<3, 1>::kCtas == 2 &&
+  static_assert(Cfg<2, 4>::kCtas == 3 && Cfg<2, 8>::kCtas == 2 && Cfg<2, 16>::kCtas == 2 && Cfg<3, 1>::kCtas == 2 &&
                     Cfg<3, 16>::kCtas == 2 && Cfg<4, 8>::kCtas == 2 && Cfg<4, 16>::kCtas == 1,
                 "keep ctas_per_sm in step with Cfg");
-  if (bits == 2 && g <= 8) return 3;
+  if (bits == 2 && g <= 4) return 3;
   return (bits == 4 && g >= 16) ? 1 : 2;
 }
 
