@@ -15,8 +15,8 @@ import math
 import torch
 
 from . import _lib
-from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_CAPACITY, STATUS_CTX_OVERFLOW,  # noqa: F401
-                   STATUS_META_OVERFLOW, STATUS_NONFINITE, STATUS_TIMEOUT, WushkvError)
+from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_BAD_PAGE, STATUS_CAPACITY,  # noqa: F401
+                   STATUS_CTX_OVERFLOW, STATUS_META_OVERFLOW, STATUS_NONFINITE, STATUS_TIMEOUT, WushkvError)
 
 HEAD_DIM = 128
 
@@ -48,15 +48,35 @@ def _dtype_code(t):
 
 
 class PackedCache:
-    """Caller-owned packed KV cache of one layer (codes + fp16 meta), see wushkv_cache."""
+    """Caller-owned packed KV cache of one layer (codes + fp16 meta), see wushkv_cache.
+
+    Contiguous: tensors [batch, Hkv, capacity, ...].  Paged (page_size given): pools
+    [num_pages, Hkv, page_size, ...] and an int32 block table [batch, capacity // page_size]
+    whose row b lists the pages of sequence b in order."""
 
     def __init__(self, batch, num_kv_heads, capacity, kind=QUEST_INT, bits=2, clip_alpha=0.0,
-                 rank_lo=2, rank_hi=125, device="cuda", tensors=None):
+                 rank_lo=2, rank_hi=125, device="cuda", tensors=None, page_size=None, num_pages=None,
+                 block_table=None):
         self.batch, self.num_kv_heads, self.capacity = int(batch), int(num_kv_heads), int(capacity)
         self.kind, self.bits = int(kind), int(bits)
         self.clip_alpha, self.rank_lo, self.rank_hi = float(clip_alpha), int(rank_lo), int(rank_hi)
+        self.page_size = None if page_size is None else int(page_size)
+        self.block_table = None
         m = 1 if self.kind == QUEST_INT else 2
-        shp = (self.batch, self.num_kv_heads, self.capacity)
+        if self.page_size is None:
+            shp = (self.batch, self.num_kv_heads, self.capacity)
+        else:
+            if self.capacity % self.page_size:
+                raise ValueError("capacity must be a multiple of page_size")
+            self.pages_per_seq = self.capacity // self.page_size
+            self.num_pages = int(num_pages if num_pages is not None else self.batch * self.pages_per_seq)
+            if block_table is None:     # sequence b owns pages b * pages_per_seq ... in order
+                block_table = torch.arange(self.batch * self.pages_per_seq, dtype=torch.int32).view(
+                    self.batch, self.pages_per_seq)
+            if tuple(block_table.shape) != (self.batch, self.pages_per_seq) or block_table.dtype != torch.int32:
+                raise ValueError("block_table must be int32 [batch, capacity // page_size]")
+            self.block_table = block_table.to(device if tensors is None else tensors["k_codes"].device).contiguous()
+            shp = (self.num_pages, self.num_kv_heads, self.page_size)
         if tensors is None:
             self.k_codes = torch.zeros(shp + (16 * self.bits,), dtype=torch.uint8, device=device)
             self.v_codes = torch.zeros_like(self.k_codes)
@@ -78,9 +98,13 @@ class PackedCache:
 
     def desc(self) -> _lib.CacheDesc:
         qp = _lib.QuantParams(self.kind, self.bits, self.clip_alpha, self.rank_lo, self.rank_hi)
+        if self.page_size is None:
+            paging = (None, 0, 0, 0)
+        else:
+            paging = (self.block_table.data_ptr(), self.pages_per_seq, self.page_size, self.num_pages)
         return _lib.CacheDesc(self.k_codes.data_ptr(), self.v_codes.data_ptr(), self.k_meta.data_ptr(),
                               self.v_meta.data_ptr(), self.batch, self.num_kv_heads, self.capacity,
-                              HEAD_DIM, qp)
+                              HEAD_DIM, qp, *paging)
 
     def tensors(self):
         return {"k_codes": self.k_codes, "v_codes": self.v_codes, "k_meta": self.k_meta, "v_meta": self.v_meta}

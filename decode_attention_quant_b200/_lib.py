@@ -30,6 +30,7 @@ STATUS_NONFINITE = 2
 STATUS_META_OVERFLOW = 4
 STATUS_CTX_OVERFLOW = 8
 STATUS_TIMEOUT = 16
+STATUS_BAD_PAGE = 32
 
 # every symbol include/wushkv.h declares
 EXPORTS = (
@@ -53,7 +54,9 @@ class CacheDesc(ctypes.Structure):
                 ("k_meta", ctypes.c_void_p), ("v_meta", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("head_dim", ctypes.c_int32),
-                ("qp", QuantParams)]
+                ("qp", QuantParams),
+                ("block_table", ctypes.c_void_p), ("pages_per_seq", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
 
 
 class WushkvError(RuntimeError):

@@ -53,6 +53,14 @@ int check_cache(const wushkv_cache* c, bool quantizing) {
     if (c->qp.rank_lo >= c->qp.rank_hi) return WUSHKV_ERR_INVALID;
     if (c->qp.rank_lo > 2 || c->qp.rank_hi < WUSHKV_HEAD_DIM - 3) return WUSHKV_ERR_UNSUPPORTED;
   }
+  if (c->block_table != nullptr) {      // paged pools: see wushkv_cache
+    const int p = c->page_size;
+    if (p < 16 || p > 4096 || (p & (p - 1)) != 0) return WUSHKV_ERR_INVALID;
+    if (c->pages_per_seq <= 0 || c->num_pages <= 0) return WUSHKV_ERR_INVALID;
+    if ((int64_t)c->pages_per_seq * p != c->capacity) return WUSHKV_ERR_INVALID;
+    if ((int64_t)c->num_pages * c->num_kv_heads * p > (int64_t)1 << 40) return WUSHKV_ERR_INVALID;
+    if (!aligned(c->block_table, 4)) return WUSHKV_ERR_MISALIGNED;
+  }
   if (!c->k_codes || !c->v_codes || !c->k_meta || !c->v_meta) return WUSHKV_ERR_INVALID;
   if (!aligned(c->k_codes, 16) || !aligned(c->v_codes, 16)) return WUSHKV_ERR_MISALIGNED;
   if (!aligned(c->k_meta, 4) || !aligned(c->v_meta, 4)) return WUSHKV_ERR_MISALIGNED;

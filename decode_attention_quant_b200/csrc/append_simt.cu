@@ -26,6 +26,7 @@ struct RowArgs {
   uint8_t* codes;          // [B][Hkv][T][16 bits]
   uint16_t* meta;          // [B][Hkv][T][m]
   int capacity;
+  CacheRows rows;          // (sequence, head, position) -> row, contiguous or paged
   double alpha;
   int rank_lo, rank_hi;
   int32_t* status;
@@ -102,11 +103,13 @@ __global__ void __launch_bounds__(kRows) append_rows_kernel(RowArgs a) {
 
   const int b = f / a.n_new, t = f - b * a.n_new;
   const int pos = __ldg(a.start_pos + b) + t;
-  const bool store = pos >= 0 && pos < a.capacity;
-  const size_t row = ((size_t)b * a.num_kv_heads + h) * a.capacity + (store ? pos : 0);
+  const bool in_cap = pos >= 0 && pos < a.capacity;
+  const long long rr = in_cap ? a.rows.row(b, h, pos) : 0;
+  const bool store = in_cap && rr >= 0;
+  const size_t row = store ? (size_t)rr : 0;
   uint8_t* dst = store ? a.codes + row * (16 * BITS) : nullptr;
   uint16_t m0 = 0, m1 = 0;
-  int32_t flags = store ? 0 : WUSHKV_STATUS_CAPACITY;
+  int32_t flags = !in_cap ? WUSHKV_STATUS_CAPACITY : store ? 0 : WUSHKV_STATUS_BAD_PAGE;
   if (KIND == WUSHKV_QUEST_INT) {
     quest_quantize<BITS>(ld, a.alpha, dst, m0, flags);
   } else {
@@ -165,6 +168,7 @@ cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new
   a.n_new = n_new;
   a.start_pos = start_pos;
   a.capacity = c.capacity;
+  a.rows = CacheRows::of(c);
   a.alpha = c.qp.clip_alpha;
   a.rank_lo = c.qp.rank_lo;
   a.rank_hi = c.qp.rank_hi;

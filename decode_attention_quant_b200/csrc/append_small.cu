@@ -29,6 +29,7 @@ struct SmallArgs {
   const __nv_bfloat16* k;           // [B*n_new][Hkv][128]
   const __nv_bfloat16* v;
   int num_kv_heads, total_rows, n_new, capacity;
+  CacheRows rows;                   // (sequence, head, position) -> row, contiguous or paged
   const int32_t* start_pos;
   const float* tk;                  // [Hkv][128][128] or nullptr
   uint8_t* k_codes;
@@ -204,9 +205,12 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
     const int f = f0 + r;
     const int b = f / a.n_new, t = f - b * a.n_new;
     const int pos = __ldg(a.start_pos + b) + t;
-    const bool store = pos >= 0 && pos < a.capacity;
-    if (!store) flags |= WUSHKV_STATUS_CAPACITY;
-    const size_t row = ((size_t)b * a.num_kv_heads + h) * a.capacity + (store ? pos : 0);
+    const bool in_cap = pos >= 0 && pos < a.capacity;
+    const long long rr = in_cap ? a.rows.row(b, h, pos) : 0;
+    const bool store = in_cap && rr >= 0;
+    if (!in_cap) flags |= WUSHKV_STATUS_CAPACITY;
+    else if (!store) flags |= WUSHKV_STATUS_BAD_PAGE;
+    const size_t row = store ? (size_t)rr : 0;
     if (side == 0) quantize_group_warp<BITS, KIND>(xk[r], a, store, row, a.k_codes, a.k_meta, flags);
     else quantize_group_warp<BITS, KIND>(xv[r], a, store, row, a.v_codes, a.v_meta, flags);
   }
@@ -242,6 +246,7 @@ cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_ne
   a.total_rows = c.batch * n_new;
   a.n_new = n_new;
   a.capacity = c.capacity;
+  a.rows = CacheRows::of(c);
   a.start_pos = start_pos;
   a.tk = Tk;
   a.k_codes = c.k_codes;

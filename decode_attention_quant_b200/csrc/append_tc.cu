@@ -48,6 +48,7 @@ constexpr int kSmemBytes = kOffBar + 256 + 1024;     // + barriers, TMEM address
 
 struct TcArgs {
   int num_kv_heads, total_rows, n_new, capacity;
+  CacheRows rows;          // (sequence, head, position) -> row, contiguous or paged
   int tiles_per_head, ctas_per_head;
   const int32_t* start_pos;
   const float* tk;
@@ -112,9 +113,12 @@ __device__ __forceinline__ void quantize_store(Loader& ld, const TcArgs& a, int 
   if (f >= 0) {
     const int b = f / a.n_new, t = f - b * a.n_new;
     const int pos = __ldg(a.start_pos + b) + t;
-    store = pos >= 0 && pos < a.capacity;
-    if (!store) flags |= WUSHKV_STATUS_CAPACITY;
-    row = ((size_t)b * a.num_kv_heads + h) * a.capacity + (store ? pos : 0);
+    const bool in_cap = pos >= 0 && pos < a.capacity;
+    const long long rr = in_cap ? a.rows.row(b, h, pos) : 0;
+    store = in_cap && rr >= 0;
+    if (!in_cap) flags |= WUSHKV_STATUS_CAPACITY;
+    else if (!store) flags |= WUSHKV_STATUS_BAD_PAGE;
+    row = store ? (size_t)rr : 0;
   }
   uint8_t* dst = store ? codes + row * (16 * BITS) : nullptr;
   uint16_t m0 = 0, m1 = 0;
@@ -380,6 +384,7 @@ cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, 
   a.total_rows = c.batch * n_new;
   a.n_new = n_new;
   a.capacity = c.capacity;
+  a.rows = CacheRows::of(c);
   a.tiles_per_head = (a.total_rows + kRowsPerTile - 1) / kRowsPerTile;
   cudaError_t e = cudaSuccess;
   const int sms = num_sms(&e);

@@ -108,6 +108,8 @@ struct DecArgs {
   float scale_log2;        // softmax scale * log2(e)
   float* ws;               // [B][Hq][S][132]
   int32_t* status;
+  CacheRows rows;          // (sequence, head, position) -> row, contiguous or paged
+  int box_rows;            // rows of one code box: the tile (contiguous) or min(page, tile)
 };
 
 struct Misc {
@@ -349,8 +351,27 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
         const int s = i % S;
         const int t0 = (tile0 + i) * kTile;
         mbar_arrive_expect_tx(&ms->full[s], 2 * kTile * C::kCode);
-        tma_load_3d(stage + s * C::kStage, &kmap, &ms->full[s], 0, t0, (int)pair);
-        tma_load_3d(stage + s * C::kStage + kTile * C::kCode, &vmap, &ms->full[s], 0, t0, (int)pair);
+        if (a.rows.block_table == nullptr) {
+          tma_load_3d(stage + s * C::kStage, &kmap, &ms->full[s], 0, t0, (int)pair);
+          tma_load_3d(stage + s * C::kStage + kTile * C::kCode, &vmap, &ms->full[s], 0, t0, (int)pair);
+        } else {
+          // one box per page the tile touches ([page * Hkv + h][row in page][byte]); rows
+          // past the capacity or in a page outside the pool come from an out-of-range
+          // coordinate and arrive as zeros
+          const int nb = kTile / a.box_rows;
+          const int oob = a.rows.num_pages * a.hkv;
+          for (int sb = 0; sb < nb; ++sb) {
+            const int t = t0 + sb * a.box_rows;
+            int page = -1;
+            if (t < a.capacity) page = __ldg(a.rows.block_table + (size_t)b * a.rows.pages_per_seq + (t >> a.rows.page_shift));
+            const bool in = page >= 0 && page < a.rows.num_pages;
+            const int c1 = in ? (t & ((1 << a.rows.page_shift) - 1)) : 0;
+            const int c2 = in ? page * a.hkv + kv : oob;
+            const int off = sb * a.box_rows * C::kCode;
+            tma_load_3d(stage + s * C::kStage + off, &kmap, &ms->full[s], 0, c1, c2);
+            tma_load_3d(stage + s * C::kStage + kTile * C::kCode + off, &vmap, &ms->full[s], 0, c1, c2);
+          }
+        }
         ++issued;
       };
       auto score_mma = [&]() {
@@ -408,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
 #pragma unroll
     for (int h = 0; h < G; ++h) { m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; o[h] = 0.f; }
     uint32_t kmeta[2] = {0u, 0u}, vmeta[2] = {0u, 0u};
+    bool page_ok[2] = {true, true};         // the tile's rows r, r + 128 sit in valid pages
     float c1[G], c2[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { c1[h] = ms->c1[h]; c2[h] = ms->c2[h]; }
@@ -417,12 +439,17 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
     auto widen_k = [&](int i) {
       const int s = i % S;
       const int t = (tile0 + i) * kTile + r;
-      const size_t mrow = pair * a.capacity + t;
 #pragma unroll
       for (int j = 0; j < 2; ++j)
         if (t + kHalf * j < L) {
-          kmeta[j] = load_meta<KIND>(a.k_meta, mrow + kHalf * j);
-          vmeta[j] = load_meta<KIND>(a.v_meta, mrow + kHalf * j);
+          const long long mrow = a.rows.row(b, kv, t + kHalf * j);
+          page_ok[j] = mrow >= 0;
+          if (mrow >= 0) {
+            kmeta[j] = load_meta<KIND>(a.k_meta, (size_t)mrow);
+            vmeta[j] = load_meta<KIND>(a.v_meta, (size_t)mrow);
+          } else {
+            report(a.status, WUSHKV_STATUS_BAD_PAGE);
+          }
         }
       ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->full[s], (i / S) & 1, abort));
       if (ok) {
@@ -470,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
     for (int i = 0; i < n; ++i) {
       const int u = i & 1;
       const int tb = (tile0 + i) * kTile + r;
-      const bool valid[2] = {tb < L, tb + kHalf < L};
+      const bool valid[2] = {tb < L && page_ok[0], tb + kHalf < L && page_ok[1]};
       float ks[2], kz[2], vs[2], vz[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -691,13 +718,14 @@ __global__ void __launch_bounds__(kHeadDim) combine_log2_kernel(const float* __r
   out[bh * kHeadDim + c] = l > 0.f ? o / l : 0.f;
 }
 
-// Tensor map over one side's codes: [pairs][capacity][16*BITS bytes], boxes of a tile's
-// 256 rows, swizzled as code_swizzle describes.
+// Tensor map over one side's codes: [planes][rows][16*BITS bytes] (planes = sequence x
+// head rows of `rows` positions, or page x head), boxes of box_rows rows, swizzled as
+// code_swizzle describes.
 template <int BITS>
-bool code_map(CUtensorMap* m, const uint8_t* base, int capacity, int pairs) {
-  const uint64_t dims[3] = {(uint64_t)(16 * BITS), (uint64_t)capacity, (uint64_t)pairs};
-  const uint64_t strides[2] = {(uint64_t)(16 * BITS), (uint64_t)capacity * (16 * BITS)};
-  const uint32_t box[3] = {(uint32_t)(16 * BITS), (uint32_t)kTile, 1};
+bool code_map(CUtensorMap* m, const uint8_t* base, int rows, int planes, int box_rows) {
+  const uint64_t dims[3] = {(uint64_t)(16 * BITS), (uint64_t)rows, (uint64_t)planes};
+  const uint64_t strides[2] = {(uint64_t)(16 * BITS), (uint64_t)rows * (16 * BITS)};
+  const uint32_t box[3] = {(uint32_t)(16 * BITS), (uint32_t)box_rows, 1};
   const CUtensorMapSwizzle sw = BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
                                 : BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
                                             : CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -711,7 +739,11 @@ cudaError_t launch_g(const DecArgs& a, int batch, float* out, cudaStream_t strea
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   CUtensorMap km, vm;
-  if (!code_map<BITS>(&km, a.k_codes, a.capacity, batch * a.hkv) || !code_map<BITS>(&vm, a.v_codes, a.capacity, batch * a.hkv))
+  // contiguous: [B * Hkv][capacity][bytes]; paged: [num_pages * Hkv][page_size][bytes]
+  const bool paged = a.rows.block_table != nullptr;
+  const int rows = paged ? (1 << a.rows.page_shift) : a.capacity;
+  const int planes = paged ? a.rows.num_pages * a.hkv : batch * a.hkv;
+  if (!code_map<BITS>(&km, a.k_codes, rows, planes, a.box_rows) || !code_map<BITS>(&vm, a.v_codes, rows, planes, a.box_rows))
     return cudaErrorInvalidValue;
   dim3 grid(a.num_splits, a.hkv, batch);
   kern<<<grid, kThreads, C::kSmem, stream>>>(km, vm, a);
@@ -790,6 +822,8 @@ cudaError_t launch_decode_attention(const wushkv_cache& c, const float* q_t, int
   a.scale_log2 = softmax_scale * kLog2e;
   a.ws = static_cast<float*>(workspace);
   a.status = status;
+  a.rows = CacheRows::of(c);
+  a.box_rows = c.block_table != nullptr ? (c.page_size < kTile ? c.page_size : kTile) : kTile;
   switch (c.qp.bits) {
     case 2: return launch_bits<2>(a, c.qp.kind, c.batch, out, stream);
     case 3: return launch_bits<3>(a, c.qp.kind, c.batch, out, stream);

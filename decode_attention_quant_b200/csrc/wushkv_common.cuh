@@ -45,6 +45,33 @@ __device__ __forceinline__ uint4 ld_global_nc_v4(const void* p) {
   return r;
 }
 
+// Row of the codes / meta arrays that holds position t of sequence b, KV head h, in the
+// contiguous layout ([batch][Hkv][capacity]) or the paged one ([num_pages][Hkv][page_size],
+// page from the block table); -1 when the block table points outside the pool.
+struct CacheRows {
+  const int32_t* block_table;   // nullptr: contiguous
+  int pages_per_seq, page_shift, num_pages, hkv, capacity;
+
+  static CacheRows of(const wushkv_cache& c) {
+    CacheRows r{};
+    r.block_table = c.block_table;
+    r.pages_per_seq = c.pages_per_seq;
+    r.num_pages = c.num_pages;
+    r.hkv = c.num_kv_heads;
+    r.capacity = c.capacity;
+    int shift = 0;
+    while (c.block_table != nullptr && (1 << shift) < c.page_size) ++shift;
+    r.page_shift = shift;
+    return r;
+  }
+  __device__ __forceinline__ long long row(int b, int h, int t) const {
+    if (block_table == nullptr) return ((long long)b * hkv + h) * capacity + t;
+    const int page = __ldg(block_table + (size_t)b * pages_per_seq + (t >> page_shift));
+    if (page < 0 || page >= num_pages) return -1;
+    return (((long long)page * hkv + h) << page_shift) + (t & ((1 << page_shift) - 1));
+  }
+};
+
 // Two bf16 packed in a 32-bit word -> two fp32 (exact).
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

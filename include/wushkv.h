@@ -57,6 +57,8 @@ typedef enum {
 #define WUSHKV_STATUS_META_OVERFLOW 4  /* a step/scale/zero overflowed fp16 (stored as Inf) */
 #define WUSHKV_STATUS_CTX_OVERFLOW 8   /* ctx_len[b] > capacity: clamped to capacity */
 #define WUSHKV_STATUS_TIMEOUT 16       /* an internal pipeline wait gave up; output unspecified */
+#define WUSHKV_STATUS_BAD_PAGE 32      /* a block-table entry outside [0, num_pages): that row was
+                                          not written (append) or was left out (decode) */
 
 /* Quantizer family [ai4s 3-5], [abs]:
  *  QUEST_INT  - QuEST-INT-style symmetric RMS-clipped grid (the quantizer of the
@@ -94,7 +96,16 @@ typedef struct {
  *   Keys are stored in the transformed basis x = T_k k [ai4s 5]; values are stored
  *   as given, since their transform is folded into the model weights [ai4s 5],
  *   [blog flowchart].  Code pointers must be 16-byte aligned, meta pointers
- *   4-byte aligned. */
+ *   4-byte aligned.
+ * Paged layout (an addition of this library for serving engines that allocate the
+ * cache in pages; the pages do not describe one): with block_table != NULL the four
+ * buffers are pools of num_pages pages, codes [num_pages][num_kv_heads][page_size]
+ * [16*bits] and meta [num_pages][num_kv_heads][page_size][m]; position t of sequence b
+ * is row t % page_size of page block_table[b * pages_per_seq + t / page_size].
+ * page_size is a power of two in [16, 4096] and capacity = pages_per_seq * page_size.
+ * block_table is int32 device memory, caller-owned and never modified; entries
+ * outside [0, num_pages) are skipped with WUSHKV_STATUS_BAD_PAGE.  With block_table ==
+ * NULL the three paging fields are ignored. */
 typedef struct {
   uint8_t* k_codes;
   uint8_t* v_codes;
@@ -105,6 +116,10 @@ typedef struct {
   int32_t capacity;    /* T_max, tokens per sequence */
   int32_t head_dim;    /* must be 128 */
   wushkv_quant_params qp;
+  const int32_t* block_table;   /* NULL: contiguous layout; else [batch][pages_per_seq] */
+  int32_t pages_per_seq;
+  int32_t page_size;
+  int32_t num_pages;
 } wushkv_cache;
 
 /* Key transform + clipped quantization + bit-packing + append.

@@ -305,3 +305,19 @@ def decode_attention_pair(k_codes, k_meta, v_codes, v_meta, q_rows, softmax_scal
         p /= np.sum(p)
         out[i] = p @ v_hat
     return out
+
+
+# ------------------------------------------------------------------- paged layout
+def gather_paged(pool, block_table, page_size):
+    """Contiguous [B, Hkv, pages_per_seq * page_size, ...] copy of a paged pool
+    [num_pages, Hkv, page_size, ...]: position t of sequence b is row t % page_size of
+    page block_table[b, t // page_size].  (The paged layout is a serving-engine
+    convention of this library, not a step of the method.)"""
+    pool = np.asarray(pool)
+    bt = np.asarray(block_table)
+    b, pps = bt.shape
+    out = np.empty((b, pool.shape[1], pps * page_size) + pool.shape[3:], dtype=pool.dtype)
+    for s in range(b):
+        for p in range(pps):
+            out[s, :, p * page_size:(p + 1) * page_size] = pool[bt[s, p]]
+    return out

@@ -124,3 +124,34 @@ def test_decode_rejects_bad_arguments():
     assert call(out=0x3004) == _lib.ERR_MISALIGNED
     assert call(ctx=0x2002) == _lib.ERR_MISALIGNED
     assert call(st=0x5002) == _lib.ERR_MISALIGNED
+
+
+PAGED_BAD = [
+    (dict(block_table=0x50000, pages_per_seq=4, page_size=48, num_pages=16, capacity=192), _lib.ERR_INVALID),
+    (dict(block_table=0x50000, pages_per_seq=4, page_size=8, num_pages=16, capacity=32), _lib.ERR_INVALID),
+    (dict(block_table=0x50000, pages_per_seq=4, page_size=64, num_pages=16, capacity=200), _lib.ERR_INVALID),
+    (dict(block_table=0x50000, pages_per_seq=0, page_size=64, num_pages=16, capacity=0), _lib.ERR_INVALID),
+    (dict(block_table=0x50000, pages_per_seq=4, page_size=64, num_pages=0, capacity=256), _lib.ERR_INVALID),
+    (dict(block_table=0x50002, pages_per_seq=4, page_size=64, num_pages=16, capacity=256), _lib.ERR_MISALIGNED),
+]
+
+
+@pytest.mark.parametrize("fields,code", PAGED_BAD)
+def test_paged_layout_checks(fields, code):
+    """Paged caches: page size a power of two in [16, 4096], capacity = pages x page size,
+    a non-empty pool and an aligned block table; rejected before any launch."""
+    d = _desc(capacity=fields.pop("capacity"))
+    for k, v in fields.items():
+        setattr(d, k, v)
+    lib = dq.library()
+    assert lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 1) == 0
+    vp = ctypes.c_void_p
+    rc = lib.wushkv_decode_attention(ctypes.byref(d), vp(0x60000), 4, vp(0x70000), 0.1, vp(0x80000),
+                                     vp(0x90000), 1 << 20, 1, vp(0), vp(0))
+    assert rc == code
+
+
+def test_paged_layout_accepted():
+    d = _desc(capacity=256)
+    d.block_table, d.pages_per_seq, d.page_size, d.num_pages = 0x50000, 4, 64, 16
+    assert dq.library().wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 1) > 0
