@@ -347,6 +347,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
       int issued = 0;
       // a tile's K and V code rows, one 3-D box each ([pair][token][byte], swizzled);
       // rows past the capacity arrive as zeros, rows past the context are never used
+      // paged caches: page of position t (-1 past the capacity)
+      auto page_at = [&](int t) {
+        return t < a.capacity ? __ldg(a.rows.block_table + (size_t)b * a.rows.pages_per_seq + (t >> a.rows.page_shift))
+                              : -1;
+      };
+      int pf_tile = -1, pf_page = -1;
       auto load = [&](int i) {
         const int s = i % S;
         const int t0 = (tile0 + i) * kTile;
@@ -362,14 +368,17 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
           const int oob = a.rows.num_pages * a.hkv;
           for (int sb = 0; sb < nb; ++sb) {
             const int t = t0 + sb * a.box_rows;
-            int page = -1;
-            if (t < a.capacity) page = __ldg(a.rows.block_table + (size_t)b * a.rows.pages_per_seq + (t >> a.rows.page_shift));
+            const int page = (nb == 1 && pf_tile == i) ? pf_page : page_at(t);
             const bool in = page >= 0 && page < a.rows.num_pages;
             const int c1 = in ? (t & ((1 << a.rows.page_shift) - 1)) : 0;
             const int c2 = in ? page * a.hkv + kv : oob;
             const int off = sb * a.box_rows * C::kCode;
             tma_load_3d(stage + s * C::kStage + off, &kmap, &ms->full[s], 0, c1, c2);
             tma_load_3d(stage + s * C::kStage + kTile * C::kCode + off, &vmap, &ms->full[s], 0, c1, c2);
+          }
+          if (nb == 1 && i + 1 < n) {        // the next tile's page, read while this one loads
+            pf_tile = i + 1;
+            pf_page = page_at((tile0 + i + 1) * kTile);
           }
         }
         ++issued;
@@ -430,6 +439,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
     for (int h = 0; h < G; ++h) { m_run[h] = -CUDART_INF_F; l_run[h] = 0.f; z_run[h] = 0.f; o[h] = 0.f; }
     uint32_t kmeta[2] = {0u, 0u}, vmeta[2] = {0u, 0u};
     bool page_ok[2] = {true, true};         // the tile's rows r, r + 128 sit in valid pages
+    // paged caches: this thread's two meta rows for the next tile, looked up one tile
+    // ahead so the block-table load is off the meta load's path
+    long long next_row[2] = {0, 0};
+    auto lookup_rows = [&](int i) {
+      if (a.rows.block_table == nullptr || i >= n) return;
+      const int t = (tile0 + i) * kTile + r;
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        next_row[j] = t + kHalf * j < L ? a.rows.row(b, kv, t + kHalf * j) : -1;
+    };
     float c1[G], c2[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { c1[h] = ms->c1[h]; c2[h] = ms->c2[h]; }
@@ -439,10 +458,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
     auto widen_k = [&](int i) {
       const int s = i % S;
       const int t = (tile0 + i) * kTile + r;
+      long long rows_i[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        rows_i[j] = a.rows.block_table == nullptr ? a.rows.row(b, kv, t + kHalf * j) : next_row[j];
+      lookup_rows(i + 1);
 #pragma unroll
       for (int j = 0; j < 2; ++j)
         if (t + kHalf * j < L) {
-          const long long mrow = a.rows.row(b, kv, t + kHalf * j);
+          const long long mrow = rows_i[j];
           page_ok[j] = mrow >= 0;
           if (mrow >= 0) {
             kmeta[j] = load_meta<KIND>(a.k_meta, (size_t)mrow);
@@ -490,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
       fence_proxy_async_smem();
     };
 
+    lookup_rows(0);
     if (n > 0) {
       widen_k(0);
       widen_v(0);
