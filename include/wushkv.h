@@ -136,9 +136,12 @@ typedef struct {
  *                  NULL means identity (the keys are taken as already transformed,
  *                  which is how the quantizer is tested on exact fp32 inputs).
  *   status       : optional int32 (device).
- * The transform runs on the tensor cores with Tk split exactly into three bf16
- * parts (products exact, fp32 accumulation); the quantizer works on the fp32
- * result.  Values never pass through the transform. */
+ * Routing: bf16 calls of at most 64 token rows (batch * n_new) take a latency
+ * kernel (FFMA transform, one warp per 128-value group); larger bf16 calls run the
+ * transform on the tensor cores with Tk split exactly into three bf16 parts
+ * (products exact, fp32 accumulation); fp32 inputs take an FFMA kernel.  In every
+ * case the quantizer works on the fp32 transform result and values never pass
+ * through the transform. */
 WUSHKV_API int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const void* v_new,
                            int32_t in_dtype, int32_t n_new, const int32_t* start_pos,
                            const float* Tk, int32_t* status, void* stream);

@@ -51,6 +51,12 @@ Readings:
   R11 positions >= capacity are not written and set status bit 1.
   R12 the value side uses the same quantizer kind, bits and parameters as the
       key side, on the untransformed value.
+  R13 chunked forward ([ai4s] paragraph 3: sequences run in 16-token forward
+      chunks): the chunk's n_q tokens are appended to the cache first, then query i
+      of the chunk (0-based) sits at position ctx - n_q + i, ctx = min(ctx_len,
+      capacity), and attends every cached position up to and including its own,
+      all read from the packed cache.  A query whose position is negative gives an
+      all-zero row (R10).
 """
 import numpy as np
 
@@ -304,6 +310,34 @@ def decode_attention_pair(k_codes, k_meta, v_codes, v_meta, q_rows, softmax_scal
         p = np.exp(s - np.max(s))
         p /= np.sum(p)
         out[i] = p @ v_hat
+    return out
+
+
+def chunk_attention(cache, q_t, ctx_len, softmax_scale, kind, bits, num_kv_heads):
+    """Causal attention of a chunk of n_q queries per sequence over the packed cache
+    (R8, R9, R10, R13).  q_t: [B, n_q, Hq, 128] transformed queries; ctx_len counts the
+    cached tokens including the chunk's own.  Returns float64 [B, n_q, Hq, 128]."""
+    q_t = np.asarray(q_t, dtype=np.float64)
+    bsz, nq, hq, d = q_t.shape
+    g = hq // num_kv_heads
+    capacity = cache["k_codes"].shape[2]
+    out = np.zeros((bsz, nq, hq, d))
+    for b in range(bsz):
+        ctx = min(max(int(ctx_len[b]), 0), capacity)
+        for kv in range(num_kv_heads):
+            k_hat = dequant_groups(unpack_codes(cache["k_codes"][b, kv, :ctx], bits),
+                                   cache["k_meta"][b, kv, :ctx], kind, bits)
+            v_hat = dequant_groups(unpack_codes(cache["v_codes"][b, kv, :ctx], bits),
+                                   cache["v_meta"][b, kv, :ctx], kind, bits)
+            for i in range(nq):
+                n = ctx - nq + i + 1          # positions 0 .. ctx - n_q + i
+                if n <= 0:
+                    continue
+                for h in range(kv * g, (kv + 1) * g):
+                    s = softmax_scale * (k_hat[:n] @ q_t[b, i, h])
+                    p = np.exp(s - np.max(s))
+                    p /= np.sum(p)
+                    out[b, i, h] = p @ v_hat[:n]
     return out
 
 

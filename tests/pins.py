@@ -322,6 +322,74 @@ def check_decode_special(orc):
             np.testing.assert_allclose(out[b, h], vh[h // 2].mean(axis=0), rtol=1e-12, atol=1e-12)
 
 
+def check_chunk_bruteforce(orc):
+    """Chunk attention (R13) against per-query windows written out by hand: query i of
+    a chunk of n_q sees positions 0 .. ctx - n_q + i of its KV head."""
+    kind, bits = 0, 2
+    cache = _small_cache(orc, kind, bits, ctx=12)
+    rng = np.random.default_rng(31)
+    hq, hkv, nq = 4, 2, 5
+    q = rng.standard_normal((2, nq, hq, 128))
+    ctx = [12, 3]                      # sequence 1: the first two queries precede position 0
+    tau = 1 / math.sqrt(128)
+    got = orc.chunk_attention(cache, q, ctx, tau, kind, bits, hkv)
+    half = 1 << (bits - 1)
+    for b in range(2):
+        for kv in range(hkv):
+            kh, vh = [], []
+            for side, dst in (("k", kh), ("v", vh)):
+                for t in range(ctx[b]):
+                    codes = bits_of_lsb_first(cache[f"{side}_codes"][b, kv, t], bits)
+                    delta = float(np.uint16(cache[f"{side}_meta"][b, kv, t, 0]).view(np.float16))
+                    dst.append([(c - half + 0.5) * delta for c in codes])
+            for i in range(nq):
+                last = ctx[b] - nq + i          # the query's own position
+                for h in range(kv * 2, kv * 2 + 2):
+                    if last < 0:
+                        assert np.all(got[b, i, h] == 0)
+                        continue
+                    s = [tau * sum(q[b, i, h, c] * kh[t][c] for c in range(128)) for t in range(last + 1)]
+                    mx = max(s)
+                    p = [math.exp(v - mx) for v in s]
+                    den = sum(p)
+                    o = [sum(p[t] * vh[t][c] for t in range(last + 1)) / den for c in range(128)]
+                    np.testing.assert_allclose(got[b, i, h], o, rtol=1e-10, atol=1e-10)
+
+
+def check_chunk_special(orc):
+    """Chunk attention invariants: its last query is the decode query at the same
+    context (decode is pinned by brute force above); a query cannot see the positions
+    after its own; a chunk query at position 0 returns the first value row."""
+    kind, bits = 1, 3
+    cache = _small_cache(orc, kind, bits)
+    rng = np.random.default_rng(37)
+    hq, hkv, nq = 4, 2, 16
+    q = rng.standard_normal((2, nq, hq, 128))
+    tau = 1 / math.sqrt(128)
+    ctx = [40, 17]
+    out = orc.chunk_attention(cache, q, ctx, tau, kind, bits, hkv)
+    dec = orc.decode_attention(cache, q[:, nq - 1], ctx, tau, kind, bits, hkv)
+    np.testing.assert_allclose(out[:, nq - 1], dec, rtol=1e-13, atol=1e-13)
+    # sequence 0: query i sits at position 24 + i.  Overwrite positions 32 .. 39 (those
+    # of queries 8 .. 15): queries 0..7 keep their outputs, queries 8 onwards change.
+    first = 40 - nq + 8
+    c2 = {k: v.copy() for k, v in cache.items()}
+    c2["k_codes"][0, :, first:40] ^= 0x5A
+    c2["v_codes"][0, :, first:40] ^= 0x3C
+    out2 = orc.chunk_attention(c2, q, ctx, tau, kind, bits, hkv)
+    assert np.array_equal(out2[0, :8], out[0, :8])
+    assert np.array_equal(out2[1], out[1])
+    for i in range(8, nq):
+        assert not np.allclose(out2[0, i], out[0, i]), i
+    # sequence of 16 tokens, chunk of 16: query 0 sees position 0 only
+    out3 = orc.chunk_attention(cache, q, [nq, nq], tau, kind, bits, hkv)
+    for b in range(2):
+        v0 = orc.dequant_groups(orc.unpack_codes(cache["v_codes"][b, :, 0], bits),
+                                cache["v_meta"][b, :, 0], kind, bits)
+        for h in range(hq):
+            np.testing.assert_allclose(out3[b, 0, h], v0[h // 2], rtol=1e-14, atol=1e-14)
+
+
 def check_append_positions(orc):
     cache = orc.empty_cache(2, 1, 10, 0, 2)
     x = np.ones((2, 3, 1, 128))
@@ -341,6 +409,6 @@ ALL_PINS = [
     check_fp16_rounding, check_quest_step, check_quest_codes_bruteforce, check_quest_degenerate,
     check_affine_bruteforce, check_affine_degenerate, check_pack_golden, check_transform,
     check_unquantized_invariance, check_decode_bruteforce, check_decode_special,
-    check_append_positions,
+    check_chunk_bruteforce, check_chunk_special, check_append_positions,
 ]
 

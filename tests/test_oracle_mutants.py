@@ -121,6 +121,28 @@ def _decode_wrong_group(cache, q_t, ctx, tau, kind, bits, hkv):
     return _orig["decode_attention"](cache, q[:, perm], ctx, tau, kind, bits, hkv)[:, np.argsort(perm)]
 
 
+def _chunk_exclusive(cache, q_t, ctx, tau, kind, bits, hkv):
+    """The query does not see its own position."""
+    q = np.asarray(q_t, np.float64)
+    nq = q.shape[1]
+    return np.stack([orc.decode_attention(cache, q[:, i], [int(n) - nq + i for n in ctx], tau, kind, bits, hkv)
+                     for i in range(nq)], axis=1)
+
+
+def _chunk_not_causal(cache, q_t, ctx, tau, kind, bits, hkv):
+    """Every query of the chunk sees the whole context."""
+    q = np.asarray(q_t, np.float64)
+    return np.stack([orc.decode_attention(cache, q[:, i], ctx, tau, kind, bits, hkv)
+                     for i in range(q.shape[1])], axis=1)
+
+
+def _chunk_positions_from_start(cache, q_t, ctx, tau, kind, bits, hkv):
+    """Query i placed at position i instead of ctx - n_q + i."""
+    q = np.asarray(q_t, np.float64)
+    return np.stack([orc.decode_attention(cache, q[:, i], [min(i + 1, int(n)) for n in ctx], tau, kind, bits, hkv)
+                     for i in range(q.shape[1])], axis=1)
+
+
 MUTANTS = {
     "transform_keys_transposed": {"transform_keys": _transform_keys_transposed},
     "transform_query_wrong_group": {"transform_query": _transform_query_wrong_group},
@@ -138,6 +160,9 @@ MUTANTS = {
     "decode_scale_wrong": {"decode_attention": _decode_scale_twice},
     "decode_unnormalized": {"decode_attention": _decode_unnormalized},
     "decode_wrong_group": {"decode_attention": _decode_wrong_group},
+    "chunk_exclusive_window": {"chunk_attention": _chunk_exclusive},
+    "chunk_not_causal": {"chunk_attention": _chunk_not_causal},
+    "chunk_positions_from_start": {"chunk_attention": _chunk_positions_from_start},
 }
 
 
