@@ -8,6 +8,7 @@ runs in the library's kernels.  PyTorch provides device memory and streams.
     quantize_append(cache, k_new, v_new, start_pos, tk)          # keys post-RoPE
     q_t = transform_query(q, tk_inv_t, num_kv_heads)
     out = decode_attention(cache, q_t, ctx_len)
+    out = chunk_attention(cache, q_t_chunk, ctx_len)              # [B, n_q, Hq, 128], causal
 """
 import ctypes
 import math
@@ -21,7 +22,8 @@ from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_BAD_PAGE, STATUS_CA
 HEAD_DIM = 128
 
 __all__ = ["PackedCache", "quantize_append", "transform_query", "decode_attention",
-           "decode_attention_noalloc", "decode_workspace_bytes", "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
+           "decode_attention_noalloc", "decode_workspace_bytes", "chunk_attention", "chunk_workspace_bytes",
+           "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
 
 
 def library():
@@ -201,4 +203,38 @@ def decode_attention_noalloc(cache: PackedCache, q_t, ctx_len, softmax_scale=Non
         raise WushkvError(rc, f"wushkv_decode_attention_noalloc: needs {decode_workspace_bytes(cache, hq, num_splits)} "
                               f"bytes of scratch, the fixed array holds {_lib.DECODE_STATIC_SCRATCH_BYTES}")
     _lib.check(rc, "wushkv_decode_attention_noalloc")
+    return out
+
+
+def chunk_workspace_bytes(cache: PackedCache, num_q_heads, n_q, num_splits=0) -> int:
+    d = cache.desc()
+    n = library().wushkv_chunk_workspace_bytes(ctypes.byref(d), int(num_q_heads), int(n_q), int(num_splits))
+    if n == 0:
+        raise WushkvError(_lib.ERR_INVALID, "wushkv_chunk_workspace_bytes")
+    return int(n)
+
+
+def chunk_attention(cache: PackedCache, q_t, ctx_len, softmax_scale=None, out=None, workspace=None,
+                    num_splits=0, status=None, stream=None):
+    """Causal attention of n_q chunk queries per sequence over the packed cache;
+    q_t fp32 [B, n_q, Hq, 128] (query i at position ctx_len - n_q + i), returns the
+    same shape."""
+    if q_t.dtype != torch.float32 or q_t.dim() != 4 or q_t.shape[0] != cache.batch or q_t.shape[3] != HEAD_DIM \
+            or not q_t.is_contiguous():
+        raise ValueError("q_t must be contiguous float32 [B, n_q, Hq, 128]")
+    if ctx_len.dtype != torch.int32 or ctx_len.numel() != cache.batch:
+        raise ValueError("ctx_len must be int32 [B]")
+    n_q, hq = int(q_t.shape[1]), int(q_t.shape[2])
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(HEAD_DIM)
+    if out is None:
+        out = torch.empty(q_t.shape, dtype=torch.float32, device=q_t.device)
+    if workspace is None:
+        workspace = torch.empty(chunk_workspace_bytes(cache, hq, n_q, num_splits), dtype=torch.uint8,
+                                device=q_t.device)
+    d = cache.desc()
+    rc = library().wushkv_chunk_attention(ctypes.byref(d), _ptr(q_t), n_q, hq, _ptr(ctx_len), float(softmax_scale),
+                                          _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          int(num_splits), _ptr(status), _stream(q_t.device, stream))
+    _lib.check(rc, "wushkv_chunk_attention")
     return out

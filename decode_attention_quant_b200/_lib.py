@@ -31,6 +31,7 @@ STATUS_META_OVERFLOW = 4
 STATUS_CTX_OVERFLOW = 8
 STATUS_TIMEOUT = 16
 STATUS_BAD_PAGE = 32
+MAX_CHUNK = 16          # WUSHKV_MAX_CHUNK
 
 # every symbol include/wushkv.h declares
 EXPORTS = (
@@ -39,6 +40,8 @@ EXPORTS = (
     "wushkv_decode_workspace_bytes",
     "wushkv_decode_attention",
     "wushkv_decode_attention_noalloc",
+    "wushkv_chunk_workspace_bytes",
+    "wushkv_chunk_attention",
     "wushkv_strerror",
     "wushkv_version",
 )
@@ -87,6 +90,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_decode_attention.restype = ctypes.c_int
     lib.wushkv_decode_attention_noalloc.argtypes = [cp, vp, i32, vp, ctypes.c_float, vp, i32, vp, vp]
     lib.wushkv_decode_attention_noalloc.restype = ctypes.c_int
+    lib.wushkv_chunk_workspace_bytes.argtypes = [cp, i32, i32, i32]
+    lib.wushkv_chunk_workspace_bytes.restype = sz
+    lib.wushkv_chunk_attention.argtypes = [cp, vp, i32, i32, vp, ctypes.c_float, vp, vp, sz, i32, vp, vp]
+    lib.wushkv_chunk_attention.restype = ctypes.c_int
     lib.wushkv_strerror.argtypes = [ctypes.c_int]
     lib.wushkv_strerror.restype = ctypes.c_char_p
     lib.wushkv_version.argtypes = []

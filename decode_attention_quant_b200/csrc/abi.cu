@@ -119,6 +119,36 @@ int wushkv_transform_query(const void* q, int32_t q_dtype, int32_t batch, int32_
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 
+size_t wushkv_chunk_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads, int32_t n_q,
+                                    int32_t num_splits) {
+  if (check_cache(cache, false) != WUSHKV_OK) return 0;
+  if (check_heads(num_q_heads, cache->num_kv_heads) != WUSHKV_OK) return 0;
+  if (n_q < 1 || n_q > WUSHKV_MAX_CHUNK || num_splits < 0 || num_splits > 4096) return 0;
+  return wushkv::chunk_workspace_bytes(*cache, num_q_heads, n_q, num_splits);
+}
+
+int wushkv_chunk_attention(const wushkv_cache* cache, const float* q_t, int32_t n_q, int32_t num_q_heads,
+                           const int32_t* ctx_len, float softmax_scale, float* out, void* workspace,
+                           size_t workspace_bytes, int32_t num_splits, int32_t* status, void* stream) {
+  int rc = check_cache(cache, false);
+  if (rc != WUSHKV_OK) return rc;
+  rc = check_heads(num_q_heads, cache->num_kv_heads);
+  if (rc != WUSHKV_OK) return rc;
+  if (n_q < 1 || n_q > WUSHKV_MAX_CHUNK) return WUSHKV_ERR_INVALID;
+  if (!q_t || !ctx_len || !out || !workspace) return WUSHKV_ERR_INVALID;
+  if ((const void*)q_t == (const void*)out) return WUSHKV_ERR_INVALID;
+  if (num_splits < 0 || num_splits > 4096) return WUSHKV_ERR_INVALID;
+  if (!std::isfinite(softmax_scale)) return WUSHKV_ERR_INVALID;
+  if (!aligned(q_t, 16) || !aligned(out, 16) || !aligned(workspace, 16) || !aligned(ctx_len, 4))
+    return WUSHKV_ERR_MISALIGNED;
+  if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
+  if (workspace_bytes < wushkv::chunk_workspace_bytes(*cache, num_q_heads, n_q, num_splits))
+    return WUSHKV_ERR_WORKSPACE;
+  cudaError_t e = wushkv::launch_chunk_attention(*cache, q_t, n_q, num_q_heads, ctx_len, softmax_scale, out,
+                                                 workspace, num_splits, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
+}
+
 size_t wushkv_decode_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads, int32_t num_splits) {
   if (check_cache(cache, false) != WUSHKV_OK) return 0;
   if (check_heads(num_q_heads, cache->num_kv_heads) != WUSHKV_OK) return 0;

@@ -207,6 +207,39 @@ WUSHKV_API int wushkv_decode_attention_noalloc(const wushkv_cache* cache, const 
                                     int32_t num_q_heads, const int32_t* ctx_len, float softmax_scale,
                                     float* out, int32_t num_splits, int32_t* status, void* stream);
 
+/* Largest number of queries per sequence that wushkv_chunk_attention takes. */
+#define WUSHKV_MAX_CHUNK 16
+
+/* Bytes of workspace needed for wushkv_chunk_attention with the same cache shape,
+ * num_q_heads, n_q and num_splits.  Returns 0 for invalid arguments.  Host only. */
+WUSHKV_API size_t wushkv_chunk_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads, int32_t n_q,
+                                    int32_t num_splits);
+
+/* Causal attention of a chunk of n_q queries per sequence over the packed cache
+ * ([ai4s 3]: perplexity runs feed each sequence in 16-token forward chunks).  The
+ * chunk's tokens must already be appended (wushkv_quantize_append), so every key and
+ * value is read in packed form.  With ctx = min(ctx_len[b], capacity), query i of
+ * sequence b sits at position ctx - n_q + i and attends positions 0 .. ctx - n_q + i:
+ *   s_t = softmax_scale * q_t[b][i][h] . k_hat_t,
+ *   out[b][i][h] = sum_t softmax(s)_t * v_hat_t   (KV head h / g).
+ * A query whose position is negative (ctx < n_q - i) gives a zero row.
+ *   q_t        : fp32 [batch][n_q][num_q_heads][128], each query mapped by
+ *                wushkv_transform_query (batch * n_q rows); 16-byte aligned.
+ *   n_q        : 1 .. WUSHKV_MAX_CHUNK.
+ *   ctx_len    : int32 [batch] (device), cached tokens including the chunk; values
+ *                > capacity are clamped (WUSHKV_STATUS_CTX_OVERFLOW).
+ *   out        : fp32 [batch][n_q][num_q_heads][128]; may not alias q_t.
+ *   workspace  : at least wushkv_chunk_workspace_bytes() bytes, 16-byte aligned.
+ *   num_splits : splits of the prefix (positions before the chunk); 0 = automatic.
+ * The positions before the chunk run through the decode kernel with the chunk's
+ * queries folded into the head group (at most 16 rows per KV head per pass, so
+ * ceil(n_q * g / 16) passes over the prefix); the chunk's own positions take a
+ * small causal kernel that also merges the two.  Errors as wushkv_decode_attention. */
+WUSHKV_API int wushkv_chunk_attention(const wushkv_cache* cache, const float* q_t, int32_t n_q,
+                           int32_t num_q_heads, const int32_t* ctx_len, float softmax_scale, float* out,
+                           void* workspace, size_t workspace_bytes, int32_t num_splits, int32_t* status,
+                           void* stream);
+
 /* Static text for a wushkv_error code, or the last CUDA error text for WUSHKV_ERR_CUDA
  * on the calling thread. */
 WUSHKV_API const char* wushkv_strerror(int code);

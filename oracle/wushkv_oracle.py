@@ -23,7 +23,8 @@ paragraph 5; [blog] flowchart); a clipped per-token scalar quantizer, QuEST-INT 
 OSCAR-style percentile-clipped affine ([ai4s] paragraphs 3-5; [abs]); 2-bit KV
 caches served with grouped-query attention ([ai4s] paragraph 5).  What the pages
 leave open is taken in its plainest reading; each reading is named where it is
-used (R1..R12 below) and listed in the design notes.
+used (R1..R12 and R18 below; R13..R17 concern the input generator and
+the parity rules, not the oracle) and listed in the design notes.
 
 Readings:
   R1  x = T_k k with column vectors; T_k stored row-major, x_i = sum_j T_ij k_j.
@@ -51,7 +52,7 @@ Readings:
   R11 positions >= capacity are not written and set status bit 1.
   R12 the value side uses the same quantizer kind, bits and parameters as the
       key side, on the untransformed value.
-  R13 chunked forward ([ai4s] paragraph 3: sequences run in 16-token forward
+  R18 chunked forward ([ai4s] paragraph 3: sequences run in 16-token forward
       chunks): the chunk's n_q tokens are appended to the cache first, then query i
       of the chunk (0-based) sits at position ctx - n_q + i, ctx = min(ctx_len,
       capacity), and attends every cached position up to and including its own,
@@ -315,7 +316,7 @@ def decode_attention_pair(k_codes, k_meta, v_codes, v_meta, q_rows, softmax_scal
 
 def chunk_attention(cache, q_t, ctx_len, softmax_scale, kind, bits, num_kv_heads):
     """Causal attention of a chunk of n_q queries per sequence over the packed cache
-    (R8, R9, R10, R13).  q_t: [B, n_q, Hq, 128] transformed queries; ctx_len counts the
+    (R8, R9, R10, R18).  q_t: [B, n_q, Hq, 128] transformed queries; ctx_len counts the
     cached tokens including the chunk's own.  Returns float64 [B, n_q, Hq, 128]."""
     q_t = np.asarray(q_t, dtype=np.float64)
     bsz, nq, hq, d = q_t.shape

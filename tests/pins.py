@@ -323,7 +323,7 @@ def check_decode_special(orc):
 
 
 def check_chunk_bruteforce(orc):
-    """Chunk attention (R13) against per-query windows written out by hand: query i of
+    """Chunk attention (R18) against per-query windows written out by hand: query i of
     a chunk of n_q sees positions 0 .. ctx - n_q + i of its KV head."""
     kind, bits = 0, 2
     cache = _small_cache(orc, kind, bits, ctx=12)

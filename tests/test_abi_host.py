@@ -155,3 +155,52 @@ def test_paged_layout_accepted():
     d = _desc(capacity=256)
     d.block_table, d.pages_per_seq, d.page_size, d.num_pages = 0x50000, 4, 64, 16
     assert dq.library().wushkv_decode_workspace_bytes(ctypes.byref(d), 4, 1) > 0
+
+
+def test_chunk_workspace_and_argument_checks():
+    lib = dq.library()
+    d = _desc()
+    # layout: prefix lengths, the decode pass's own output, folded queries and split partials
+    # of each pass (16 rows per KV head per pass), each rounded up to 64 floats
+    def floats(hq, n_q, splits):
+        r64 = lambda n: -(-n // 64) * 64
+        rows = n_q * (hq // 2)
+        total = r64(2) + r64(2 * 2 * 16 * 128)
+        passes = []
+        while rows > 0:
+            gf = 1
+            while gf < min(rows, 16):
+                gf *= 2
+            passes.append(gf)
+            rows -= 16
+        total += sum(r64(2 * 2 * gf * 128) for gf in passes)
+        total += sum(r64(2 * 2 * gf * splits * 132) for gf in passes)
+        return total
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 16, 3) == 4 * floats(4, 16, 3) == 301312
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 3, 3) == 4 * floats(4, 3, 3) == 100096
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 0, 0) == 0
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 17, 0) == 0
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 6, 4, 0) == 0
+    need = lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 16, 0)
+    assert need > 0
+    f = lib.wushkv_chunk_attention
+    ok = (ctypes.byref(d), 0x1000, 16, 4, 0x2000, 0.1, 0x3000, 0x4000, need, 0, None, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["c", "q", "nq", "hq", "ctx", "scale", "out", "ws", "wsb", "ns", "st", "stream"]
+        for k, v in kw.items():
+            args[names.index(k)] = v
+        return f(*args)
+
+    assert call(wsb=need - 1) == _lib.ERR_WORKSPACE
+    assert call(nq=0) == _lib.ERR_INVALID
+    assert call(nq=17) == _lib.ERR_INVALID
+    assert call(q=None) == _lib.ERR_INVALID
+    assert call(out=0x1000) == _lib.ERR_INVALID
+    assert call(hq=6) == _lib.ERR_UNSUPPORTED
+    assert call(ns=-1) == _lib.ERR_INVALID
+    assert call(scale=float("nan")) == _lib.ERR_INVALID
+    assert call(q=0x1008) == _lib.ERR_MISALIGNED
+    assert call(ws=0x4008) == _lib.ERR_MISALIGNED
+    assert call(ctx=0x2002) == _lib.ERR_MISALIGNED
