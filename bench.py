@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synth import gen  # noqa: E402
-from synth.configs import QWEN8B_DECODE, QWEN8B_SWEEP  # noqa: E402
+from synth.configs import QWEN8B_DECODE, QWEN8B_SWEEP, quest  # noqa: E402
 
 METRIC = "2-bit KV decode-attn HBM GB/s (% of peak) & quant-append tokens/s, 1×B200"
 TAU = 1.0 / math.sqrt(128)
@@ -81,6 +81,25 @@ def _peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def _int8_tensor_peak():
+    """Dense int8 tensor peak in TOP/s: the measured bf16 burst GEMM rate times the
+    nominal int8/bf16 ratio (4.5 / 2.25), else the fallback bf16 figure times the same."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return 2.0 * float(d["bf16_tflops"]), "measured bf16 burst x 2 (nominal int8 / bf16)"
+    return 2.0 * 1590.0, "fallback bf16 x 2 (nominal int8 / bf16)"
+
+
+def chunk_flops(batch, n_q, num_q_heads, ctx):
+    """Algorithmic FLOPs of one chunk-attention call: for every (query row, cached
+    position) pair, a 128-long score dot product and a 128-long value accumulation, two
+    FLOPs per multiply-add (the causal mask's savings on the last n_q positions ignored)."""
+    return 4 * 128 * batch * n_q * num_q_heads * ctx
 
 
 # --------------------------------------------------------------------- byte counts
@@ -350,6 +369,8 @@ def run_ours(args, rank, world, local):
     paged = bench_paged_decode(dq, cache, q_t, ctx, out, args, world)
     # quantize-append throughput: 2048-token chunk per sequence, QuEST 2-bit
     app = bench_append(dq, device, args, world)
+    # causal 16-query chunk attention over the packed cache
+    chunk = bench_chunk(dq, device, args, world)
     st = int(status.item())
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -368,6 +389,7 @@ def run_ours(args, rank, world, local):
                      "alg_bytes_per_launch": dec_alg, "launch_ms": round(dec_ms, 5)},
         "append": app,
         "paged_decode": paged,
+        "chunk_attention": chunk,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -416,6 +438,61 @@ def bench_paged_decode(dq, cache, q_t, ctx, out, args, world, page_size=256):
     return {"page_size": page_size, "ms": round(ms, 5), "GB/s": round(world * by / (ms * 1e-3) / 1e9, 1),
             "frac_of_peak": round(by / (ms * 1e-3) / 1e9 / _peaks()[0], 4), "output_equals_contiguous": same,
             "l2": "inputs larger than L2"}
+
+
+def bench_chunk(dq, device, args, world):
+    """Causal chunk attention (16 queries per sequence over the packed cache) on two
+    shapes: a Qwen3-32B-shaped layer at context 8192 (cache above L2) and the last
+    chunk of a 2048-token Qwen3-8B-shaped sequence, QuEST 2-bit, L2 flushed before
+    each rep.  Bytes: the cache up to ctx read once, queries in and outputs out."""
+    n_q = 16
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    peak, _ = _peaks()
+    res = []
+    for name, batch, hq, hkv, ctx in (("qwen3_32b_layer_b32_ctx8192_chunk16_quest2", 32, 64, 8, 8192),
+                                      ("qwen3_8b_b16_ctx2048_chunk16_quest2", 16, 32, 8, 2048)):
+        qs = quest(2)
+        c = gen.random_cache(batch, hkv, ctx, qs.kind, qs.bits, seed=ctx, device=device)
+        cache = dq.PackedCache(batch, hkv, ctx, qs.kind, qs.bits, qs.clip_alpha, tensors=c)
+        q = torch.randn(batch, n_q, hq, 128, generator=torch.Generator(device=device).manual_seed(1),
+                        device=device)
+        ctx_t = torch.full((batch,), ctx, dtype=torch.int32, device=device)
+        out = torch.empty_like(q)
+        ws = torch.empty(dq.chunk_workspace_bytes(cache, hq, n_q), dtype=torch.uint8, device=device)
+        for _ in range(max(3, args.warmup)):
+            dq.chunk_attention(cache, q, ctx_t, TAU, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(max(5, args.steps)):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            torch.cuda.nvtx.range_push(f"chunk_attention_{name}")   # lets a profiler select these launches
+            a.record(stream)
+            dq.chunk_attention(cache, q, ctx_t, TAU, out=out, workspace=ws)
+            b.record(stream)
+            torch.cuda.nvtx.range_pop()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = max_over_ranks(statistics.median(times), world)
+        by = batch * hkv * ctx * 2 * group_bytes(qs) + 2 * q.numel() * 4
+        gbs = by / (ms * 1e-3) / 1e9
+        passes = -(-n_q * (hq // hkv) // 16)
+        fl = chunk_flops(batch, n_q, hq, ctx)
+        tpeak, tkind = _int8_tensor_peak()
+        tops = fl / (ms * 1e-3) / 1e12
+        res.append({"workload": name, "n_q": n_q, "ms": round(ms, 5), "GB/s": round(world * gbs, 1),
+                    "frac_of_peak": round(gbs / peak, 4), "alg_bytes": by, "prefix_passes": passes,
+                    "roofline": {"bound": "tensor", "achieved": round(tops, 1), "peak": round(tpeak, 1),
+                                 "unit": "TFLOP/s", "frac": round(tops / tpeak, 4), "peak_kind": tkind,
+                                 "flops_per_call": fl, "hbm_floor_ms": round(by / (peak * 1e9) * 1e3, 5),
+                                 "tensor_floor_ms": round(fl / (tpeak * 1e12) * 1e3, 5)},
+                    "launches_per_call": 2 + 2 * passes,
+                    "queries_per_s": round(world * batch * n_q * hq / (ms * 1e-3), 1),
+                    "l2": "flushed (512 MB write) before each rep"})
+        del c, cache, q, out, ws
+    return res
 
 
 def bench_append(dq, device, args, world):

@@ -44,3 +44,13 @@ def test_two_gloo_ranks_agree_on_max_and_reference_runs_on_rank0_only():
     assert [g[:3] for g in got] == [(0, 2, 0), (1, 2, 1)]
     assert all(g[3] == pytest.approx(11.5) for g in got)
     assert got[1][4] is None                     # rank 1 of the reference arm does no work
+
+
+def test_chunk_roofline_helpers():
+    """FLOP count of the chunk-attention sub-benchmark and the int8 tensor peak it is
+    compared with (host logic only)."""
+    import bench
+    # Qwen3-32B-shaped layer: 32 sequences x 16 queries x 64 heads x 8192 positions, 512 FLOPs each
+    assert bench.chunk_flops(32, 16, 64, 8192) == 512 * 32 * 16 * 64 * 8192 == 137438953472
+    peak, kind = bench._int8_tensor_peak()
+    assert peak > 1000.0 and "x 2" in kind
