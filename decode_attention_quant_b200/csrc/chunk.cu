@@ -306,10 +306,6 @@ size_t chunk_workspace_bytes(const wushkv_cache& c, int num_q_heads, int n_q, in
   return (size_t)make_plan(c, num_q_heads, n_q, num_splits).floats * sizeof(float);
 }
 
-int chunk_launches(const wushkv_cache& c, int num_q_heads, int n_q) {
-  return 2 + 2 * make_plan(c, num_q_heads, n_q, 1).passes;
-}
-
 cudaError_t launch_chunk_attention(const wushkv_cache& c, const float* q_t, int n_q, int num_q_heads,
                                    const int32_t* ctx_len, float softmax_scale, float* out, void* workspace,
                                    int num_splits, int32_t* status, cudaStream_t stream) {

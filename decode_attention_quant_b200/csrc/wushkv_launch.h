@@ -28,9 +28,8 @@ cudaError_t launch_decode_attention(const wushkv_cache& c, const float* q_t, int
                                     void* workspace, int num_splits, int32_t* status,
                                     cudaStream_t stream);
 
-// Chunk attention (chunk.cu): workspace bytes, kernel launches per call, and the call.
+// Chunk attention (chunk.cu): workspace bytes and the call.
 size_t chunk_workspace_bytes(const wushkv_cache& c, int num_q_heads, int n_q, int num_splits);
-int chunk_launches(const wushkv_cache& c, int num_q_heads, int n_q);
 cudaError_t launch_chunk_attention(const wushkv_cache& c, const float* q_t, int n_q, int num_q_heads,
                                    const int32_t* ctx_len, float softmax_scale, float* out, void* workspace,
                                    int num_splits, int32_t* status, cudaStream_t stream);

@@ -23,7 +23,7 @@ paragraph 5; [blog] flowchart); a clipped per-token scalar quantizer, QuEST-INT 
 OSCAR-style percentile-clipped affine ([ai4s] paragraphs 3-5; [abs]); 2-bit KV
 caches served with grouped-query attention ([ai4s] paragraph 5).  What the pages
 leave open is taken in its plainest reading; each reading is named where it is
-used (R1..R12 and R18 below; R13..R17 concern the input generator and
+used (R1..R12, R18 and R19 below; R13..R17 concern the input generator and
 the parity rules, not the oracle) and listed in the design notes.
 
 Readings:
@@ -52,6 +52,12 @@ Readings:
   R11 positions >= capacity are not written and set status bit 1.
   R12 the value side uses the same quantizer kind, bits and parameters as the
       key side, on the untransformed value.
+  R19 fused RoPE ([ai4s] paragraph 5: the key transform follows RoPE): rotate-half
+      pairs (i, i + 64), k_i -> k_i cos_i - k_{i+64} sin_i and k_{i+64} -> k_{i+64}
+      cos_i + k_i sin_i for i < 64, with cos, sin read from row p (the key's
+      position) of a caller-supplied fp32 table [rows][128] (cos in the first 64
+      entries, sin in the last 64); the rotated key is not rounded before the
+      transform.
   R18 chunked forward ([ai4s] paragraph 3: sequences run in 16-token forward
       chunks): the chunk's n_q tokens are appended to the cache first, then query i
       of the chunk (0-based) sits at position ctx - n_q + i, ctx = min(ctx_len,
@@ -270,6 +276,35 @@ def quantize_append(cache, k_new, v_new, start_pos, kind, bits, clip_alpha=0.0,
                 cache[f"{side}_codes"][b, :, pos, :] = packed[b, t]
                 cache[f"{side}_meta"][b, :, pos, :] = meta[b, t]
     return status
+
+
+# ---------------------------------------------------------------------------- RoPE
+def apply_rope(k, cos, sin):
+    """Rotate-half RoPE (R19): k [..., 128]; cos, sin [..., 64] broadcast against it."""
+    k = np.asarray(k, dtype=np.float64)
+    cos = np.asarray(cos, dtype=np.float64)
+    sin = np.asarray(sin, dtype=np.float64)
+    lo, hi = k[..., :HEAD_DIM // 2], k[..., HEAD_DIM // 2:]
+    return np.concatenate([lo * cos - hi * sin, hi * cos + lo * sin], axis=-1)
+
+
+def quantize_append_rope(cache, k_pre, v_new, start_pos, rope_table, kind, bits, clip_alpha=0.0,
+                         rank_lo=2, rank_hi=125, tk=None):
+    """RoPE fused in front of the transform (R19): the key of position p = start_pos[b] + t
+    is rotated with row p of rope_table [rows >= capacity][128], then appended exactly as
+    quantize_append does.  k_pre: [B, n, Hkv, 128] pre-RoPE keys."""
+    k_pre = np.asarray(k_pre, dtype=np.float64)
+    tab = np.asarray(rope_table, dtype=np.float64)
+    capacity = cache["k_codes"].shape[2]
+    assert tab.shape[0] >= capacity and tab.shape[1] == HEAD_DIM
+    bsz, n = k_pre.shape[:2]
+    k_rot = k_pre.copy()
+    for b in range(bsz):
+        for t in range(n):
+            p = int(start_pos[b]) + t
+            if 0 <= p < capacity:             # other positions are not written (R11)
+                k_rot[b, t] = apply_rope(k_pre[b, t], tab[p, :HEAD_DIM // 2], tab[p, HEAD_DIM // 2:])
+    return quantize_append(cache, k_rot, v_new, start_pos, kind, bits, clip_alpha, rank_lo, rank_hi, tk=tk)
 
 
 # ----------------------------------------------------------------------- attention

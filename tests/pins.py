@@ -390,6 +390,77 @@ def check_chunk_special(orc):
             np.testing.assert_allclose(out3[b, 0, h], v0[h // 2], rtol=1e-14, atol=1e-14)
 
 
+def check_rope(orc):
+    """RoPE (R19): identity at angle 0; a quarter turn maps the pair (x, y) of channels
+    (i, i + 64) to (-y, x); the rotation keeps the norm; rotated dot products depend only
+    on the difference of the positions (table built here from math.cos / math.sin)."""
+    rng = np.random.default_rng(41)
+    k = rng.standard_normal((3, 128))
+    assert np.array_equal(orc.apply_rope(k, np.ones(64), np.zeros(64)), k)
+    for i in (0, 17, 63):
+        e = np.zeros(128)
+        e[i] = 1.0
+        cos, sin = np.zeros(64), np.zeros(64)
+        cos[:] = 1.0
+        cos[i], sin[i] = 0.0, 1.0                     # quarter turn of pair i only
+        out = orc.apply_rope(e, cos, sin)
+        want = np.zeros(128)
+        want[i + 64] = 1.0
+        assert np.array_equal(out, want), i
+        e2 = np.zeros(128)
+        e2[i + 64] = 1.0
+        want2 = np.zeros(128)
+        want2[i] = -1.0
+        assert np.array_equal(orc.apply_rope(e2, cos, sin), want2), i
+
+    def table_row(p, theta=1.0e6):
+        ang = [p * theta ** (-2.0 * j / 128) for j in range(64)]
+        return np.array([math.cos(a) for a in ang]), np.array([math.sin(a) for a in ang])
+    q = rng.standard_normal(128)
+    c5, s5 = table_row(5)
+    c2, s2 = table_row(2)
+    c13, s13 = table_row(13)
+    c10, s10 = table_row(10)
+    rq = orc.apply_rope(q, c5, s5)
+    np.testing.assert_allclose(np.linalg.norm(rq), np.linalg.norm(q), rtol=1e-14)
+    d1 = rq @ orc.apply_rope(k[0], c2, s2)
+    d2 = orc.apply_rope(q, c13, s13) @ orc.apply_rope(k[0], c10, s10)
+    np.testing.assert_allclose(d1, d2, rtol=1e-11, atol=1e-11)
+    assert abs(d1 - q @ k[0]) > 1e-3                  # the rotation does change the product
+
+
+def check_append_rope(orc):
+    """Fused-RoPE append (R19): an identity table gives the plain append; a table that
+    turns only position 5 by a quarter turn changes only the row written at position 5,
+    and that row equals the plain append of the key with its pairs swapped as (-y, x)."""
+    rng = np.random.default_rng(43)
+    bsz, n, hkv, cap = 2, 4, 2, 12
+    k = rng.standard_normal((bsz, n, hkv, 128)) * np.exp(rng.standard_normal(128))
+    v = rng.standard_normal((bsz, n, hkv, 128))
+    tk = np.stack([np.linalg.qr(rng.standard_normal((128, 128)))[0] for _ in range(hkv)])
+    start = [3, 8]                                    # sequence 0 writes positions 3..6, sequence 1 8..11
+    ident = np.concatenate([np.ones((cap, 64)), np.zeros((cap, 64))], axis=1)
+    for kind, bits, alpha in ((0, 2, QUEST_ALPHA[2]), (1, 3, 0.0)):
+        a = orc.empty_cache(bsz, hkv, cap, kind, bits)
+        b = orc.empty_cache(bsz, hkv, cap, kind, bits)
+        assert orc.quantize_append_rope(a, k, v, start, ident, kind, bits, alpha, tk=tk) == 0
+        assert orc.quantize_append(b, k, v, start, kind, bits, alpha, tk=tk) == 0
+        for name in a:
+            assert np.array_equal(a[name], b[name]), name
+        quarter = ident.copy()
+        quarter[5] = np.concatenate([np.zeros(64), np.ones(64)])
+        c = orc.empty_cache(bsz, hkv, cap, kind, bits)
+        assert orc.quantize_append_rope(c, k, v, start, quarter, kind, bits, alpha, tk=tk) == 0
+        swapped = k.copy()
+        swapped[0, 2] = np.concatenate([-k[0, 2, :, 64:], k[0, 2, :, :64]], axis=-1)   # position 3 + 2 = 5
+        d = orc.empty_cache(bsz, hkv, cap, kind, bits)
+        assert orc.quantize_append(d, swapped, v, start, kind, bits, alpha, tk=tk) == 0
+        for name in c:
+            assert np.array_equal(c[name], d[name]), name
+        assert not np.array_equal(c["k_codes"][0, :, 5], a["k_codes"][0, :, 5])
+        assert np.array_equal(c["v_codes"], a["v_codes"])
+
+
 def check_append_positions(orc):
     cache = orc.empty_cache(2, 1, 10, 0, 2)
     x = np.ones((2, 3, 1, 128))
@@ -409,6 +480,6 @@ ALL_PINS = [
     check_fp16_rounding, check_quest_step, check_quest_codes_bruteforce, check_quest_degenerate,
     check_affine_bruteforce, check_affine_degenerate, check_pack_golden, check_transform,
     check_unquantized_invariance, check_decode_bruteforce, check_decode_special,
-    check_chunk_bruteforce, check_chunk_special, check_append_positions,
+    check_chunk_bruteforce, check_chunk_special, check_rope, check_append_rope, check_append_positions,
 ]
 

@@ -143,6 +143,33 @@ def _chunk_positions_from_start(cache, q_t, ctx, tau, kind, bits, hkv):
                      for i in range(q.shape[1])], axis=1)
 
 
+def _rope_interleaved(k, cos, sin):
+    """Pairs (2i, 2i + 1) instead of (i, i + 64)."""
+    k = np.asarray(k, np.float64)
+    ev, od = k[..., 0::2], k[..., 1::2]
+    out = np.empty_like(k)
+    out[..., 0::2] = ev * cos - od * sin
+    out[..., 1::2] = od * cos + ev * sin
+    return out
+
+
+def _rope_wrong_sign(k, cos, sin):
+    k = np.asarray(k, np.float64)
+    lo, hi = k[..., :64], k[..., 64:]
+    return np.concatenate([lo * cos + hi * sin, hi * cos - lo * sin], axis=-1)
+
+
+def _append_rope_start_row(cache, k_pre, v_new, start_pos, tab, kind, bits, alpha=0.0, rlo=2, rhi=125, tk=None):
+    """Every row of a sequence rotated with the table row of its first position."""
+    k_pre = np.asarray(k_pre, np.float64)
+    tab = np.asarray(tab, np.float64)
+    k_rot = k_pre.copy()
+    for b in range(k_pre.shape[0]):
+        p = int(start_pos[b])
+        k_rot[b] = orc.apply_rope(k_pre[b], tab[p, :64], tab[p, 64:])
+    return orc.quantize_append(cache, k_rot, v_new, start_pos, kind, bits, alpha, rlo, rhi, tk=tk)
+
+
 MUTANTS = {
     "transform_keys_transposed": {"transform_keys": _transform_keys_transposed},
     "transform_query_wrong_group": {"transform_query": _transform_query_wrong_group},
@@ -163,6 +190,9 @@ MUTANTS = {
     "chunk_exclusive_window": {"chunk_attention": _chunk_exclusive},
     "chunk_not_causal": {"chunk_attention": _chunk_not_causal},
     "chunk_positions_from_start": {"chunk_attention": _chunk_positions_from_start},
+    "rope_interleaved_pairs": {"apply_rope": _rope_interleaved},
+    "rope_wrong_sign": {"apply_rope": _rope_wrong_sign},
+    "append_rope_start_row": {"quantize_append_rope": _append_rope_start_row},
 }
 
 
