@@ -371,6 +371,8 @@ def run_ours(args, rank, world, local):
     app = bench_append(dq, device, args, world)
     # causal 16-query chunk attention over the packed cache
     chunk = bench_chunk(dq, device, args, world)
+    # decode-step append with RoPE fused in front of the transform
+    rope_app = bench_rope_append(dq, device, args, world)
     st = int(status.item())
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -390,6 +392,7 @@ def run_ours(args, rank, world, local):
         "append": app,
         "paged_decode": paged,
         "chunk_attention": chunk,
+        "append_rope": rope_app,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -493,6 +496,42 @@ def bench_chunk(dq, device, args, world):
                     "l2": "flushed (512 MB write) before each rep"})
         del c, cache, q, out, ws
     return res
+
+
+def bench_rope_append(dq, device, args, world):
+    """Decode-step append (one token for each of 16 sequences x 8 KV heads, Qwen3-8B
+    shapes, affine 2-bit) with RoPE fused in front of the transform, against the same
+    append given post-RoPE keys: back-to-back calls between two events (inputs L2-warm)."""
+    w = QWEN8B_DECODE
+    qs = w.quant
+    cap = 4096
+    cache = dq.PackedCache(w.batch, w.num_kv_heads, cap, qs.kind, qs.bits, qs.clip_alpha, device=device)
+    tk = torch.from_numpy(gen.transforms(w)[0]).to(device)
+    table = gen.rope_table(cap, w.rope_theta).to(device)
+    sp = torch.arange(w.batch, dtype=torch.int32, device=device) * 200
+    k_pre = gen.keys(w, 0, w.batch, sp.tolist(), 1, rope=False, device=device)
+    k_post = gen.keys(w, 0, w.batch, sp.tolist(), 1, device=device)
+    v = gen.values(w, 0, w.batch, sp.tolist(), 1, device=device)
+    stream = torch.cuda.current_stream(device)
+    reps = max(50, 10 * args.steps)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b) / reps, world)
+
+    fused = timed(lambda: dq.quantize_append_rope(cache, k_pre, v, sp, table, tk))
+    plain = timed(lambda: dq.quantize_append(cache, k_post, v, sp, tk))
+    return {"workload": f"{w.name}: 1 token x 16 sequences x 8 KV heads", "fused_rope_us": round(fused * 1e3, 2),
+            "post_rope_input_us": round(plain * 1e3, 2), "calls": reps, "l2": "inputs L2-warm (back-to-back calls)"}
 
 
 def bench_append(dq, device, args, world):

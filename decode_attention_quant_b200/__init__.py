@@ -21,7 +21,7 @@ from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_BAD_PAGE, STATUS_CA
 
 HEAD_DIM = 128
 
-__all__ = ["PackedCache", "quantize_append", "transform_query", "decode_attention",
+__all__ = ["PackedCache", "quantize_append", "quantize_append_rope", "transform_query", "decode_attention",
            "decode_attention_noalloc", "decode_workspace_bytes", "chunk_attention", "chunk_workspace_bytes",
            "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
 
@@ -132,6 +132,33 @@ def quantize_append(cache: PackedCache, k_new, v_new, start_pos, tk=None, status
                                           int(k_new.shape[1]), _ptr(start_pos), _ptr(tk), _ptr(status),
                                           _stream(cache.device, stream))
     _lib.check(rc, "wushkv_quantize_append")
+
+
+def quantize_append_rope(cache: PackedCache, k_new, v_new, start_pos, rope_table, tk=None, status=None,
+                         stream=None):
+    """quantize_append with RoPE fused in front of the key transform: k_new holds pre-RoPE
+    keys; the key of position p is rotated with rope_table[p] (fp32 [rows >= capacity, 128]:
+    cos of the 64 pairs, then sin).  Decode-step appends only (bf16, B * n_new <= 64)."""
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    if k_new.dim() != 4 or k_new.shape[0] != cache.batch or k_new.shape[2] != cache.num_kv_heads \
+            or k_new.shape[3] != HEAD_DIM:
+        raise ValueError(f"k_new must be [B={cache.batch}, n, Hkv={cache.num_kv_heads}, 128]")
+    if not (k_new.is_contiguous() and v_new.is_contiguous()):
+        raise ValueError("k_new and v_new must be contiguous")
+    if start_pos.dtype != torch.int32 or start_pos.numel() != cache.batch:
+        raise ValueError("start_pos must be int32 [B]")
+    if tk is not None and (tk.dtype != torch.float32 or tuple(tk.shape) != (cache.num_kv_heads, HEAD_DIM, HEAD_DIM)
+                           or not tk.is_contiguous()):
+        raise ValueError("tk must be contiguous float32 [Hkv, 128, 128]")
+    if rope_table.dtype != torch.float32 or rope_table.dim() != 2 or rope_table.shape[1] != HEAD_DIM \
+            or not rope_table.is_contiguous():
+        raise ValueError("rope_table must be contiguous float32 [rows, 128]")
+    d = cache.desc()
+    rc = library().wushkv_quantize_append_rope(ctypes.byref(d), _ptr(k_new), _ptr(v_new), _dtype_code(k_new),
+                                               int(k_new.shape[1]), _ptr(start_pos), _ptr(tk), _ptr(rope_table),
+                                               int(rope_table.shape[0]), _ptr(status), _stream(cache.device, stream))
+    _lib.check(rc, "wushkv_quantize_append_rope")
 
 
 def transform_query(q, tk_inv_t, num_kv_heads, out=None, stream=None):

@@ -36,6 +36,7 @@ MAX_CHUNK = 16          # WUSHKV_MAX_CHUNK
 # every symbol include/wushkv.h declares
 EXPORTS = (
     "wushkv_quantize_append",
+    "wushkv_quantize_append_rope",
     "wushkv_transform_query",
     "wushkv_decode_workspace_bytes",
     "wushkv_decode_attention",
@@ -82,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     cp = ctypes.POINTER(CacheDesc)
     lib.wushkv_quantize_append.argtypes = [cp, vp, vp, i32, i32, vp, vp, vp, vp]
     lib.wushkv_quantize_append.restype = ctypes.c_int
+    lib.wushkv_quantize_append_rope.argtypes = [cp, vp, vp, i32, i32, vp, vp, vp, i32, vp, vp]
+    lib.wushkv_quantize_append_rope.restype = ctypes.c_int
     lib.wushkv_transform_query.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
     lib.wushkv_transform_query.restype = ctypes.c_int
     lib.wushkv_decode_workspace_bytes.argtypes = [cp, i32, i32]

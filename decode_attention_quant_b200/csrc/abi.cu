@@ -16,8 +16,8 @@ cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new
                                         int in_dtype, int n_new, const int32_t* start_pos,
                                         const float* Tk, int32_t* status, cudaStream_t stream);
 cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                         const int32_t* start_pos, const float* Tk, int32_t* status,
-                                         cudaStream_t stream);
+                                         const int32_t* start_pos, const float* Tk, const float* rope,
+                                         int rope_rows, int32_t* status, cudaStream_t stream);
 }
 
 namespace {
@@ -98,11 +98,30 @@ int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (in_dtype == WUSHKV_BF16 && (int64_t)cache->batch * n_new <= kSmallAppendRows)
-    e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
+    e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, nullptr, 0, status, st);
   else if (in_dtype == WUSHKV_BF16)
     e = wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
   else
     e = wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos, Tk, status, st);
+  return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
+}
+
+int wushkv_quantize_append_rope(const wushkv_cache* cache, const void* k_new, const void* v_new,
+                                int32_t in_dtype, int32_t n_new, const int32_t* start_pos, const float* Tk,
+                                const float* rope_table, int32_t rope_rows, int32_t* status, void* stream) {
+  int rc = check_cache(cache, true);
+  if (rc != WUSHKV_OK) return rc;
+  if (in_dtype != WUSHKV_BF16 && in_dtype != WUSHKV_FP32) return WUSHKV_ERR_UNSUPPORTED;
+  if (n_new <= 0 || !k_new || !v_new || !start_pos || !rope_table) return WUSHKV_ERR_INVALID;
+  if (rope_rows < cache->capacity) return WUSHKV_ERR_INVALID;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(start_pos, 4) || !aligned(rope_table, 16))
+    return WUSHKV_ERR_MISALIGNED;
+  if (Tk != nullptr && !aligned(Tk, 16)) return WUSHKV_ERR_MISALIGNED;
+  if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
+  // fused RoPE is built for decode-step appends (bf16, at most 64 token rows per call)
+  if (in_dtype != WUSHKV_BF16 || (int64_t)cache->batch * n_new > 64) return WUSHKV_ERR_UNSUPPORTED;
+  cudaError_t e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, rope_table,
+                                                       rope_rows, status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 

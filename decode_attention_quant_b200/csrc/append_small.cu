@@ -3,7 +3,8 @@
 // one KV head.  The key transform is a dot product per output channel (thread i owns
 // channel i and reads row i of T_k), then each 128-value group (key or value of one
 // row) is quantized by one warp, four values per lane, with every code decided by
-// exact threshold comparisons.
+// exact threshold comparisons.  Optionally the keys arrive before RoPE and are rotated
+// here with the caller's cos/sin table, in front of the transform.
 //
 // WUSH-KV (ai4snews summary, paragraphs 1 and 5; cere-bro page, flowchart): one key
 // transform per KV head applied online to post-RoPE keys; values already in the
@@ -32,6 +33,8 @@ struct SmallArgs {
   CacheRows rows;                   // (sequence, head, position) -> row, contiguous or paged
   const int32_t* start_pos;
   const float* tk;                  // [Hkv][128][128] or nullptr
+  const float* rope;                // [rope_rows][128] (cos | sin per position) or nullptr
+  int rope_rows;
   uint8_t* k_codes;
   uint8_t* v_codes;
   uint16_t* k_meta;
@@ -159,11 +162,11 @@ __device__ void quantize_group_warp(const float* x, const SmallArgs& a, bool sto
   }
 }
 
-template <int BITS, int KIND, bool TRANSFORM>
+template <int BITS, int KIND, bool TRANSFORM, bool ROPE>
 __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
   __shared__ __align__(16) float xk[kRows][kHeadDim];   // keys (transformed)
   __shared__ __align__(16) float xv[kRows][kHeadDim];   // values
-  __shared__ __align__(16) float kr[kRows][kHeadDim];   // raw keys (transform input)
+  __shared__ __align__(16) float kr[kRows][kHeadDim];   // raw keys (RoPE / transform input)
   const int h = blockIdx.x, f0 = blockIdx.y * kRows, tid = threadIdx.x;
   const int nrows = min(kRows, a.total_rows - f0);
   for (int e = tid; e < nrows * kHeadDim; e += kThreads) {
@@ -171,10 +174,33 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
     const size_t off = ((size_t)(f0 + r) * a.num_kv_heads + h) * kHeadDim + c;
     xv[r][c] = __bfloat162float(a.v[off]);
     const float kv = __bfloat162float(a.k[off]);
-    if (TRANSFORM) kr[r][c] = kv;
+    if (TRANSFORM || ROPE) kr[r][c] = kv;
     else xk[r][c] = kv;
   }
   __syncthreads();
+  if (ROPE) {
+    // rotate-half RoPE of each key row with the table row of its position: pair
+    // (c, c + 64) -> (x cos - y sin, y cos + x sin); a thread owns whole pairs, so the
+    // rotation can stay in place when the transform follows
+    for (int e = tid; e < nrows * (kHeadDim / 2); e += kThreads) {
+      const int r = e / (kHeadDim / 2), c = e % (kHeadDim / 2);
+      const int f = f0 + r;
+      const int b = f / a.n_new, t = f - b * a.n_new;
+      const int pos = __ldg(a.start_pos + b) + t;
+      const float x = kr[r][c], y = kr[r][c + kHeadDim / 2];
+      float rx = x, ry = y;
+      if (pos >= 0 && pos < a.rope_rows) {         // other positions are not stored
+        const float cs = __ldg(a.rope + (size_t)pos * kHeadDim + c);
+        const float sn = __ldg(a.rope + (size_t)pos * kHeadDim + kHeadDim / 2 + c);
+        rx = fmaf(x, cs, -(y * sn));
+        ry = fmaf(y, cs, x * sn);
+      }
+      float* dst = TRANSFORM ? kr[r] : xk[r];
+      dst[c] = rx;
+      dst[c + kHeadDim / 2] = ry;
+    }
+    __syncthreads();
+  }
   if (TRANSFORM) {
     // x[r][i] = sum_j T[i][j] k[r][j]: thread i reads row i of T once for every row r
     const float4* trow = reinterpret_cast<const float4*>(a.tk + ((size_t)h * kHeadDim + tid) * kHeadDim);
@@ -220,8 +246,11 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
 template <int BITS, int KIND>
 cudaError_t launch_kind(const SmallArgs& a, cudaStream_t stream) {
   dim3 grid(a.num_kv_heads, (a.total_rows + kRows - 1) / kRows);
-  if (a.tk != nullptr) append_small_kernel<BITS, KIND, true><<<grid, kThreads, 0, stream>>>(a);
-  else append_small_kernel<BITS, KIND, false><<<grid, kThreads, 0, stream>>>(a);
+  const bool tf = a.tk != nullptr, rope = a.rope != nullptr;
+  if (tf && rope) append_small_kernel<BITS, KIND, true, true><<<grid, kThreads, 0, stream>>>(a);
+  else if (tf) append_small_kernel<BITS, KIND, true, false><<<grid, kThreads, 0, stream>>>(a);
+  else if (rope) append_small_kernel<BITS, KIND, false, true><<<grid, kThreads, 0, stream>>>(a);
+  else append_small_kernel<BITS, KIND, false, false><<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -237,8 +266,8 @@ cudaError_t launch_bits(const SmallArgs& a, int bits, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                         const int32_t* start_pos, const float* Tk, int32_t* status,
-                                         cudaStream_t stream) {
+                                         const int32_t* start_pos, const float* Tk, const float* rope,
+                                         int rope_rows, int32_t* status, cudaStream_t stream) {
   SmallArgs a{};
   a.k = static_cast<const __nv_bfloat16*>(k_new);
   a.v = static_cast<const __nv_bfloat16*>(v_new);
@@ -249,6 +278,8 @@ cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_ne
   a.rows = CacheRows::of(c);
   a.start_pos = start_pos;
   a.tk = Tk;
+  a.rope = rope;
+  a.rope_rows = rope_rows;
   a.k_codes = c.k_codes;
   a.v_codes = c.v_codes;
   a.k_meta = c.k_meta;

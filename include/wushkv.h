@@ -146,6 +146,23 @@ WUSHKV_API int wushkv_quantize_append(const wushkv_cache* cache, const void* k_n
                            int32_t in_dtype, int32_t n_new, const int32_t* start_pos,
                            const float* Tk, int32_t* status, void* stream);
 
+/* wushkv_quantize_append with RoPE fused in front of the key transform ([ai4s 5]: the
+ * transform is applied to keys after RoPE).  k_new holds the keys BEFORE RoPE; the key
+ * of position p = start_pos[b] + t is rotated in rotate-half pairs (c, c + 64), c < 64:
+ *   (x, y) -> (x cos_c - y sin_c, y cos_c + x sin_c),
+ * with cos_c = rope_table[p][c] and sin_c = rope_table[p][64 + c], in fp32 and without
+ * rounding the rotated key, then transformed, quantized and appended as
+ * wushkv_quantize_append does.  Values are not rotated.
+ *   rope_table : fp32 [rope_rows][128] (device, caller-owned, 16-byte aligned), the
+ *                serving engine's cos/sin cache; rope_rows >= capacity.
+ * Built for decode-step appends: bf16 inputs and batch * n_new <= 64 token rows;
+ * other calls return WUSHKV_ERR_UNSUPPORTED (rotate first, then call
+ * wushkv_quantize_append).  Other arguments, errors and status bits as
+ * wushkv_quantize_append. */
+WUSHKV_API int wushkv_quantize_append_rope(const wushkv_cache* cache, const void* k_new, const void* v_new,
+                                int32_t in_dtype, int32_t n_new, const int32_t* start_pos, const float* Tk,
+                                const float* rope_table, int32_t rope_rows, int32_t* status, void* stream);
+
 /* Decode-query map q' = T_k^{-T} q, with T_k of the query head's KV head h / g,
  * g = num_q_heads / num_kv_heads.  Needed because keys are cached as T_k k, and
  * (T_k^{-T} q) . (T_k k) = q . k keeps the attention scores unchanged (implied by

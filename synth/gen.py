@@ -85,8 +85,9 @@ def rope_tables(positions: torch.Tensor, theta: float):
 
 
 def keys(w: Workload, b0: int, b1: int, t0, n: int, layer: int = 0, device="cpu",
-         salt: int = 0) -> torch.Tensor:
-    """Post-RoPE bf16 keys [b1-b0][n][Hkv][128] for positions t0..t0+n-1.
+         salt: int = 0, rope: bool = True) -> torch.Tensor:
+    """Post-RoPE bf16 keys [b1-b0][n][Hkv][128] for positions t0..t0+n-1 (rope=False:
+    the same draws before RoPE, rounded once to bf16).
 
     t0 is an int or a per-sequence int sequence of start positions.
     """
@@ -94,6 +95,8 @@ def keys(w: Workload, b0: int, b1: int, t0, n: int, layer: int = 0, device="cpu"
     nb = b1 - b0
     k = torch.randn((nb, n, w.num_kv_heads, _D), generator=g, device=device, dtype=torch.float64)
     k *= torch.as_tensor(key_channel_scale(w, layer), device=device)[None, None]
+    if not rope:
+        return k.to(torch.float32).to(torch.bfloat16)
     starts = torch.as_tensor(np.broadcast_to(np.asarray(t0, np.int64), (nb,)).copy(), device=device)
     pos = starts[:, None] + torch.arange(n, device=device)[None, :]
     cos, sin = rope_tables(pos, w.rope_theta)
@@ -113,6 +116,13 @@ def values(w: Workload, b0: int, b1: int, t0, n: int, layer: int = 0, device="cp
     for c in w.value_heavy:
         v[..., c] *= w.value_heavy_gain
     return v.to(torch.bfloat16)
+
+
+def rope_table(rows: int, theta: float) -> torch.Tensor:
+    """fp32 [rows][128] cos/sin cache of a serving engine: row p = cos of the 64
+    rotate-half pairs at position p, then their sin (computed in fp64, rounded once)."""
+    cos, sin = rope_tables(torch.arange(rows), theta)
+    return torch.cat([cos, sin], dim=-1).to(torch.float32).contiguous()
 
 
 def queries(w: Workload, layer: int = 0, device="cpu", salt: int = 0) -> torch.Tensor:

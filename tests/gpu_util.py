@@ -57,3 +57,45 @@ def attention_errors(got, ref):
     max_abs = float(np.max(np.abs(got - ref))) if got.size else 0.0
     rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
     return max_abs, rel_l2
+
+
+def check_key_rows(oc, gc, x, kind, bits, start, alpha):
+    """End-to-end rule for the key side of an append: oracle cache oc and GPU cache gc
+    (numpy dicts), x = the oracle's transformed keys [B, n, Hkv, 128] written at
+    start[b] + t.  Meta may differ by one fp16 ulp only where the oracle's pre-rounding
+    value lies within 1e-4 * Delta of an fp16 midpoint; codes (against the oracle's
+    quantizer given the GPU's meta) by +-1 only within 1e-4 * Delta of a threshold.
+    Returns (meta flips, code differences, values near a boundary)."""
+    bsz, n = x.shape[:2]
+    meta_flips = code_diffs = near = 0
+    for b in range(bsz):
+        sl = slice(start[b], start[b] + n)
+        om = oc["k_meta"][b, :, sl].transpose(1, 0, 2)
+        gm = gc["k_meta"][b, :, sl].transpose(1, 0, 2)
+        xo = x[b]
+        flip = np.any(om != gm, axis=-1)
+        if flip.any():
+            if kind == orc.QUEST_INT:
+                dist = fp16_midpoint_distance(orc.quest_step_prerounding(xo, bits, alpha))
+                assert np.all(dist[flip] <= 1e-4 * orc.fp16_value(om[..., 0])[flip])
+            else:
+                sp, lo = orc.affine_prerounding(xo, bits, 2, 125)
+                dd = np.minimum(fp16_midpoint_distance(sp), fp16_midpoint_distance(lo))
+                assert np.all(dd[flip] <= 1e-4 * orc.fp16_value(om[..., 0])[flip])
+            meta_flips += int(flip.sum())
+        gmv = orc.fp16_value(gm)
+        if kind == orc.QUEST_INT:
+            ref = orc.quest_codes(xo, gmv[..., 0], bits)
+            dist = quest_boundary_distance(xo, gmv[..., 0], bits)
+        else:
+            ref = orc.affine_codes(xo, gmv[..., 0], gmv[..., 1], bits)
+            dist = affine_boundary_distance(xo, gmv[..., 0], gmv[..., 1], bits)
+        step = np.broadcast_to(gmv[..., 0][..., None], dist.shape)
+        got = orc.unpack_codes(gc["k_codes"][b, :, sl].transpose(1, 0, 2), bits)
+        diff = got.astype(np.int32) - ref.astype(np.int32)
+        assert np.all(np.abs(diff) <= 1)
+        off = diff != 0
+        assert np.all(dist[off] <= 1e-4 * step[off]), "code differs away from a boundary"
+        code_diffs += int(off.sum())
+        near += int((dist <= 1e-4 * step).sum())
+    return meta_flips, code_diffs, near

@@ -204,3 +204,25 @@ def test_chunk_workspace_and_argument_checks():
     assert call(q=0x1008) == _lib.ERR_MISALIGNED
     assert call(ws=0x4008) == _lib.ERR_MISALIGNED
     assert call(ctx=0x2002) == _lib.ERR_MISALIGNED
+
+
+def test_append_rope_argument_checks():
+    lib = dq.library()
+    d = _desc()                                          # batch 2, Hkv 2, capacity 256
+    f = lib.wushkv_quantize_append_rope
+    ok = (ctypes.byref(d), 0x50000, 0x60000, 0, 4, 0x70000, None, 0x80000, 256, None, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["c", "k", "v", "dt", "n", "sp", "tk", "tab", "rows", "st", "stream"]
+        for key, val in kw.items():
+            args[names.index(key)] = val
+        return f(*args)
+
+    assert call(tab=None) == _lib.ERR_INVALID
+    assert call(rows=255) == _lib.ERR_INVALID            # the table must cover the capacity
+    assert call(tab=0x80008) == _lib.ERR_MISALIGNED
+    assert call(n=33) == _lib.ERR_UNSUPPORTED            # 66 token rows: not a decode-step append
+    assert call(dt=1) == _lib.ERR_UNSUPPORTED            # fp32 keys
+    assert call(dt=7) == _lib.ERR_UNSUPPORTED
+    assert call(n=0) == _lib.ERR_INVALID
