@@ -23,7 +23,7 @@ paragraph 5; [blog] flowchart); a clipped per-token scalar quantizer, QuEST-INT 
 OSCAR-style percentile-clipped affine ([ai4s] paragraphs 3-5; [abs]); 2-bit KV
 caches served with grouped-query attention ([ai4s] paragraph 5).  What the pages
 leave open is taken in its plainest reading; each reading is named where it is
-used (R1..R12, R18 and R19 below; R13..R17 concern the input generator and
+used (R1..R12 and R18..R20 below; R13..R17 concern the input generator and
 the parity rules, not the oracle) and listed in the design notes.
 
 Readings:
@@ -58,6 +58,12 @@ Readings:
       position) of a caller-supplied fp32 table [rows][128] (cos in the first 64
       entries, sin in the last 64); the rotated key is not rounded before the
       transform.
+  R20 structured key transforms ([ai4s] paragraph 6: cheaper structured transforms
+      are the authors' future work; Hadamard is a baseline): (a) block-diagonal T_k,
+      n/b blocks of b x b on the diagonal, block j acting on channels [j b, (j+1) b);
+      (b) T_k = H diag(s) / sqrt(128) with H the Sylvester Hadamard matrix
+      (H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]) and s a per-channel scale.  Both
+      are ordinary invertible T_k, applied by the same definition x = T_k k (R1).
   R18 chunked forward ([ai4s] paragraph 3: sequences run in 16-token forward
       chunks): the chunk's n_q tokens are appended to the cache first, then query i
       of the chunk (0-based) sits at position ctx - n_q + i, ctx = min(ctx_len,
@@ -123,6 +129,43 @@ def transform_keys(k, tk):
     for h in range(tk.shape[0]):
         x[..., h, :] = k[..., h, :] @ tk[h].T
     return x
+
+
+def block_diagonal_transform(blocks):
+    """Dense T_k [Hkv, 128, 128] of block-diagonal transforms (R20a).
+    blocks: [Hkv, 128 / b, b, b]; block j sits on rows and columns [j b, (j + 1) b)."""
+    blocks = np.asarray(blocks, dtype=np.float64)
+    hkv, nb, bs, _ = blocks.shape
+    assert nb * bs == HEAD_DIM
+    tk = np.zeros((hkv, HEAD_DIM, HEAD_DIM))
+    for h in range(hkv):
+        for j in range(nb):
+            tk[h, j * bs:(j + 1) * bs, j * bs:(j + 1) * bs] = blocks[h, j]
+    return tk
+
+
+def hadamard(n):
+    """Sylvester Hadamard matrix of order n (a power of two) (R20b)."""
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    assert h.shape[0] == n
+    return h
+
+
+def hadamard_diag_transform(scale):
+    """T_k = H diag(s) / sqrt(128) per KV head (R20b).  scale: [Hkv, 128], nonzero."""
+    s = np.asarray(scale, dtype=np.float64)
+    h = hadamard(HEAD_DIM) / np.sqrt(HEAD_DIM)
+    return np.stack([h * s[i][None, :] for i in range(s.shape[0])])
+
+
+def hadamard_diag_inverse_transpose(scale):
+    """T_k^{-T} of hadamard_diag_transform: H diag(1/s) / sqrt(128), since H / sqrt(128)
+    is symmetric and orthogonal (R2, R20b)."""
+    s = np.asarray(scale, dtype=np.float64)
+    h = hadamard(HEAD_DIM) / np.sqrt(HEAD_DIM)
+    return np.stack([h / s[i][None, :] for i in range(s.shape[0])])
 
 
 def transform_query(q, tk_inv_t, num_kv_heads):

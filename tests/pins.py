@@ -461,6 +461,39 @@ def check_append_rope(orc):
         assert np.array_equal(c["v_codes"], a["v_codes"])
 
 
+def check_structured_transforms(orc):
+    """Structured key transforms (R20): the Sylvester Hadamard matrix equals the library's
+    (scipy.linalg.hadamard) and H H^T = n I; the closed-form inverse-transpose of
+    H diag(s) / sqrt(128) equals numpy's inverse, and keeps q' . x = q . k; a
+    block-diagonal T_k applied to keys equals the per-block products written as loops."""
+    import scipy.linalg
+    for n in (1, 2, 8, 128):
+        h = orc.hadamard(n)
+        assert np.array_equal(h, scipy.linalg.hadamard(n).astype(np.float64)), n
+        assert np.array_equal(h @ h.T, n * np.eye(n)), n
+    rng = np.random.default_rng(47)
+    s = np.exp(rng.uniform(np.log(0.25), np.log(4.0), (2, 128))) * rng.choice([-1.0, 1.0], (2, 128))
+    t = orc.hadamard_diag_transform(s)
+    m = orc.hadamard_diag_inverse_transpose(s)
+    for i in range(2):
+        np.testing.assert_allclose(m[i], np.linalg.inv(t[i]).T, rtol=1e-12, atol=1e-13)
+    k = rng.standard_normal((3, 2, 128))
+    q = rng.standard_normal((3, 2, 128))
+    x = orc.transform_keys(k, t)
+    qt = orc.transform_query(q, m, 2)
+    np.testing.assert_allclose(np.sum(qt * x, axis=-1), np.sum(q * k, axis=-1), rtol=1e-11, atol=1e-11)
+    for bs in (16, 32, 64):
+        blocks = rng.standard_normal((2, 128 // bs, bs, bs))
+        tk = orc.block_diagonal_transform(blocks)
+        got = orc.transform_keys(k, tk)
+        for a in range(3):
+            for h in range(2):
+                for j in range(128 // bs):
+                    for r in range(bs):
+                        want = sum(blocks[h, j, r, c] * k[a, h, j * bs + c] for c in range(bs))
+                        assert abs(got[a, h, j * bs + r] - want) <= 1e-12 * (1 + abs(want)), (bs, a, h, j, r)
+
+
 def check_append_positions(orc):
     cache = orc.empty_cache(2, 1, 10, 0, 2)
     x = np.ones((2, 3, 1, 128))
@@ -480,6 +513,7 @@ ALL_PINS = [
     check_fp16_rounding, check_quest_step, check_quest_codes_bruteforce, check_quest_degenerate,
     check_affine_bruteforce, check_affine_degenerate, check_pack_golden, check_transform,
     check_unquantized_invariance, check_decode_bruteforce, check_decode_special,
-    check_chunk_bruteforce, check_chunk_special, check_rope, check_append_rope, check_append_positions,
+    check_chunk_bruteforce, check_chunk_special, check_rope, check_append_rope, check_structured_transforms,
+    check_append_positions,
 ]
 

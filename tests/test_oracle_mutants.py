@@ -170,6 +170,26 @@ def _append_rope_start_row(cache, k_pre, v_new, start_pos, tab, kind, bits, alph
     return orc.quantize_append(cache, k_rot, v_new, start_pos, kind, bits, alpha, rlo, rhi, tk=tk)
 
 
+def _hadamard_transposed_blocks(n):
+    """Sylvester recursion with the sign on the wrong block: [[H, -H], [H, H]]."""
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, -h], [h, h]])
+    return h
+
+
+def _hadamard_inv_t_unscaled(scale):
+    """Inverse-transpose that forgets to invert the diagonal."""
+    s = np.asarray(scale, np.float64)
+    h = orc.hadamard(128) / np.sqrt(128)
+    return np.stack([h * s[i][None, :] for i in range(s.shape[0])])
+
+
+def _block_diag_transposed(blocks):
+    """Each block placed transposed."""
+    return _orig["block_diagonal_transform"](np.swapaxes(np.asarray(blocks), -1, -2))
+
+
 MUTANTS = {
     "transform_keys_transposed": {"transform_keys": _transform_keys_transposed},
     "transform_query_wrong_group": {"transform_query": _transform_query_wrong_group},
@@ -193,6 +213,9 @@ MUTANTS = {
     "rope_interleaved_pairs": {"apply_rope": _rope_interleaved},
     "rope_wrong_sign": {"apply_rope": _rope_wrong_sign},
     "append_rope_start_row": {"quantize_append_rope": _append_rope_start_row},
+    "hadamard_wrong_sign_block": {"hadamard": _hadamard_transposed_blocks},
+    "hadamard_inverse_unscaled": {"hadamard_diag_inverse_transpose": _hadamard_inv_t_unscaled},
+    "block_diagonal_transposed": {"block_diagonal_transform": _block_diag_transposed},
 }
 
 
