@@ -494,6 +494,53 @@ def check_structured_transforms(orc):
                         assert abs(got[a, h, j * bs + r] - want) <= 1e-12 * (1 + abs(want)), (bs, a, h, j, r)
 
 
+def check_decode_pair(orc):
+    """decode_attention_pair (one sequence and KV head, used for sampled full-size checks)
+    against an explicit-loop softmax over hand-dequantized rows."""
+    kind, bits = 1, 2
+    cache = _small_cache(orc, kind, bits, ctx=9, batch=1, hkv=1)
+    rng = np.random.default_rng(53)
+    q = rng.standard_normal((2, 128))
+    tau = 0.125
+    n = 7
+    got = orc.decode_attention_pair(cache["k_codes"][0, 0, :n], cache["k_meta"][0, 0, :n], cache["v_codes"][0, 0, :n],
+                                    cache["v_meta"][0, 0, :n], q, tau, kind, bits)
+    rows = {}
+    for side in ("k", "v"):
+        rows[side] = []
+        for t in range(n):
+            codes = bits_of_lsb_first(cache[f"{side}_codes"][0, 0, t], bits)
+            sc, z = [float(np.uint16(m).view(np.float16)) for m in cache[f"{side}_meta"][0, 0, t]]
+            rows[side].append([z + c * sc for c in codes])
+    for i in range(2):
+        s = [tau * sum(q[i, c] * rows["k"][t][c] for c in range(128)) for t in range(n)]
+        mx = max(s)
+        p = [math.exp(x - mx) for x in s]
+        o = [sum(p[t] * rows["v"][t][c] for t in range(n)) / sum(p) for c in range(128)]
+        np.testing.assert_allclose(got[i], o, rtol=1e-10, atol=1e-10)
+    empty = orc.decode_attention_pair(cache["k_codes"][0, 0, :0], cache["k_meta"][0, 0, :0], cache["v_codes"][0, 0, :0],
+                                      cache["v_meta"][0, 0, :0], q, tau, kind, bits)
+    assert np.all(empty == 0)
+
+
+def check_gather_paged(orc):
+    """gather_paged against entries labelled with their page and row: position t of
+    sequence b must come from row t % page_size of page block_table[b][t // page_size]."""
+    num_pages, hkv, ps = 7, 2, 4
+    pool = np.zeros((num_pages, hkv, ps, 3), dtype=np.int64)
+    for pg in range(num_pages):
+        for h in range(hkv):
+            for r in range(ps):
+                pool[pg, h, r] = [pg, h, r]
+    bt = np.array([[5, 0, 3], [2, 6, 1]])
+    out = orc.gather_paged(pool, bt, ps)
+    assert out.shape == (2, hkv, 3 * ps, 3)
+    for b in range(2):
+        for h in range(hkv):
+            for t in range(3 * ps):
+                assert out[b, h, t].tolist() == [bt[b][t // ps], h, t % ps], (b, h, t)
+
+
 def check_append_positions(orc):
     cache = orc.empty_cache(2, 1, 10, 0, 2)
     x = np.ones((2, 3, 1, 128))
@@ -514,6 +561,6 @@ ALL_PINS = [
     check_affine_bruteforce, check_affine_degenerate, check_pack_golden, check_transform,
     check_unquantized_invariance, check_decode_bruteforce, check_decode_special,
     check_chunk_bruteforce, check_chunk_special, check_rope, check_append_rope, check_structured_transforms,
-    check_append_positions,
+    check_decode_pair, check_gather_paged, check_append_positions,
 ]
 

@@ -190,6 +190,22 @@ def _block_diag_transposed(blocks):
     return _orig["block_diagonal_transform"](np.swapaxes(np.asarray(blocks), -1, -2))
 
 
+def _pair_no_max_shift_wrong_scale(kc, km, vc, vm, q, tau, kind, bits):
+    return _orig["decode_attention_pair"](kc, km, vc, vm, q, tau * 1.25, kind, bits)
+
+
+def _gather_pages_by_modulo(pool, bt, ps):
+    """Page index taken as t % pages_per_seq instead of t // page_size."""
+    pool = np.asarray(pool)
+    bt = np.asarray(bt)
+    b, pps = bt.shape
+    out = np.empty((b, pool.shape[1], pps * ps) + pool.shape[3:], dtype=pool.dtype)
+    for s_ in range(b):
+        for t in range(pps * ps):
+            out[s_, :, t] = pool[bt[s_, t % pps], :, t % ps]
+    return out
+
+
 MUTANTS = {
     "transform_keys_transposed": {"transform_keys": _transform_keys_transposed},
     "transform_query_wrong_group": {"transform_query": _transform_query_wrong_group},
@@ -216,6 +232,8 @@ MUTANTS = {
     "hadamard_wrong_sign_block": {"hadamard": _hadamard_transposed_blocks},
     "hadamard_inverse_unscaled": {"hadamard_diag_inverse_transpose": _hadamard_inv_t_unscaled},
     "block_diagonal_transposed": {"block_diagonal_transform": _block_diag_transposed},
+    "decode_pair_scale_wrong": {"decode_attention_pair": _pair_no_max_shift_wrong_scale},
+    "gather_page_index_modulo": {"gather_paged": _gather_pages_by_modulo},
 }
 
 
