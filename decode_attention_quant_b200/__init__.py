@@ -17,11 +17,12 @@ import torch
 
 from . import _lib
 from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_BAD_PAGE, STATUS_CAPACITY,  # noqa: F401
-                   STATUS_CTX_OVERFLOW, STATUS_META_OVERFLOW, STATUS_NONFINITE, STATUS_TIMEOUT, WushkvError)
+                   STATUS_CTX_OVERFLOW, STATUS_META_OVERFLOW, STATUS_NONFINITE, STATUS_TIMEOUT,
+                   TRANSFORM_BLOCK_DIAG, TRANSFORM_DENSE, TRANSFORM_HADAMARD_DIAG, WushkvError)
 
 HEAD_DIM = 128
 
-__all__ = ["PackedCache", "quantize_append", "quantize_append_rope", "transform_query", "decode_attention",
+__all__ = ["PackedCache", "quantize_append", "quantize_append_rope", "quantize_append_structured", "transform_query", "decode_attention",
            "decode_attention_noalloc", "decode_workspace_bytes", "chunk_attention", "chunk_workspace_bytes",
            "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
 
@@ -159,6 +160,35 @@ def quantize_append_rope(cache: PackedCache, k_new, v_new, start_pos, rope_table
                                                int(k_new.shape[1]), _ptr(start_pos), _ptr(tk), _ptr(rope_table),
                                                int(rope_table.shape[0]), _ptr(status), _stream(cache.device, stream))
     _lib.check(rc, "wushkv_quantize_append_rope")
+
+
+def quantize_append_structured(cache: PackedCache, k_new, v_new, start_pos, kind, data, block=0, status=None,
+                               stream=None):
+    """quantize_append with a structured key transform (kind = TRANSFORM_BLOCK_DIAG with
+    data fp32 [Hkv, 128/block, block, block], or TRANSFORM_HADAMARD_DIAG with data = s fp32
+    [Hkv, 128], T_k = H diag(s) / sqrt(128)); decode-step appends only (bf16, B * n_new <= 64).
+    TRANSFORM_DENSE takes data as the dense T_k of quantize_append."""
+    if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and dtype")
+    if k_new.dim() != 4 or k_new.shape[0] != cache.batch or k_new.shape[2] != cache.num_kv_heads \
+            or k_new.shape[3] != HEAD_DIM:
+        raise ValueError(f"k_new must be [B={cache.batch}, n, Hkv={cache.num_kv_heads}, 128]")
+    if not (k_new.is_contiguous() and v_new.is_contiguous()):
+        raise ValueError("k_new and v_new must be contiguous")
+    if start_pos.dtype != torch.int32 or start_pos.numel() != cache.batch:
+        raise ValueError("start_pos must be int32 [B]")
+    shapes = {_lib.TRANSFORM_DENSE: (cache.num_kv_heads, HEAD_DIM, HEAD_DIM),
+              _lib.TRANSFORM_BLOCK_DIAG: (cache.num_kv_heads, HEAD_DIM // max(int(block), 1), int(block), int(block)),
+              _lib.TRANSFORM_HADAMARD_DIAG: (cache.num_kv_heads, HEAD_DIM)}
+    if int(kind) not in shapes:
+        raise ValueError("unknown transform kind")
+    if data.dtype != torch.float32 or tuple(data.shape) != shapes[int(kind)] or not data.is_contiguous():
+        raise ValueError(f"transform data must be contiguous float32 {shapes[int(kind)]}")
+    d = cache.desc()
+    rc = library().wushkv_quantize_append_structured(ctypes.byref(d), _ptr(k_new), _ptr(v_new), _dtype_code(k_new),
+                                                     int(k_new.shape[1]), _ptr(start_pos), int(kind), int(block),
+                                                     _ptr(data), _ptr(status), _stream(cache.device, stream))
+    _lib.check(rc, "wushkv_quantize_append_structured")
 
 
 def transform_query(q, tk_inv_t, num_kv_heads, out=None, stream=None):

@@ -32,11 +32,13 @@ STATUS_CTX_OVERFLOW = 8
 STATUS_TIMEOUT = 16
 STATUS_BAD_PAGE = 32
 MAX_CHUNK = 16          # WUSHKV_MAX_CHUNK
+TRANSFORM_DENSE, TRANSFORM_BLOCK_DIAG, TRANSFORM_HADAMARD_DIAG = 1, 2, 3   # wushkv_transform_kind
 
 # every symbol include/wushkv.h declares
 EXPORTS = (
     "wushkv_quantize_append",
     "wushkv_quantize_append_rope",
+    "wushkv_quantize_append_structured",
     "wushkv_transform_query",
     "wushkv_decode_workspace_bytes",
     "wushkv_decode_attention",
@@ -85,6 +87,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_quantize_append.restype = ctypes.c_int
     lib.wushkv_quantize_append_rope.argtypes = [cp, vp, vp, i32, i32, vp, vp, vp, i32, vp, vp]
     lib.wushkv_quantize_append_rope.restype = ctypes.c_int
+    lib.wushkv_quantize_append_structured.argtypes = [cp, vp, vp, i32, i32, vp, i32, i32, vp, vp, vp]
+    lib.wushkv_quantize_append_structured.restype = ctypes.c_int
     lib.wushkv_transform_query.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
     lib.wushkv_transform_query.restype = ctypes.c_int
     lib.wushkv_decode_workspace_bytes.argtypes = [cp, i32, i32]

@@ -16,8 +16,8 @@ cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new
                                         int in_dtype, int n_new, const int32_t* start_pos,
                                         const float* Tk, int32_t* status, cudaStream_t stream);
 cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                         const int32_t* start_pos, const float* Tk, const float* rope,
-                                         int rope_rows, int32_t* status, cudaStream_t stream);
+                                         const int32_t* start_pos, const float* Tk, int tkind, int tblock,
+                                         const float* rope, int rope_rows, int32_t* status, cudaStream_t stream);
 }
 
 namespace {
@@ -98,7 +98,8 @@ int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const v
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (in_dtype == WUSHKV_BF16 && (int64_t)cache->batch * n_new <= kSmallAppendRows)
-    e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, nullptr, 0, status, st);
+    e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, WUSHKV_TRANSFORM_DENSE, 0,
+                                             nullptr, 0, status, st);
   else if (in_dtype == WUSHKV_BF16)
     e = wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
   else
@@ -120,8 +121,32 @@ int wushkv_quantize_append_rope(const wushkv_cache* cache, const void* k_new, co
   if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
   // fused RoPE is built for decode-step appends (bf16, at most 64 token rows per call)
   if (in_dtype != WUSHKV_BF16 || (int64_t)cache->batch * n_new > 64) return WUSHKV_ERR_UNSUPPORTED;
-  cudaError_t e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, rope_table,
-                                                       rope_rows, status, static_cast<cudaStream_t>(stream));
+  cudaError_t e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk,
+                                                       WUSHKV_TRANSFORM_DENSE, 0, rope_table, rope_rows, status,
+                                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
+}
+
+int wushkv_quantize_append_structured(const wushkv_cache* cache, const void* k_new, const void* v_new,
+                                      int32_t in_dtype, int32_t n_new, const int32_t* start_pos, int32_t kind,
+                                      int32_t block, const float* data, int32_t* status, void* stream) {
+  if (kind == WUSHKV_TRANSFORM_DENSE) {
+    if (data == nullptr) return WUSHKV_ERR_INVALID;
+    return wushkv_quantize_append(cache, k_new, v_new, in_dtype, n_new, start_pos, data, status, stream);
+  }
+  if (kind != WUSHKV_TRANSFORM_BLOCK_DIAG && kind != WUSHKV_TRANSFORM_HADAMARD_DIAG) return WUSHKV_ERR_UNSUPPORTED;
+  if (kind == WUSHKV_TRANSFORM_BLOCK_DIAG && block != 16 && block != 32 && block != 64) return WUSHKV_ERR_UNSUPPORTED;
+  int rc = check_cache(cache, true);
+  if (rc != WUSHKV_OK) return rc;
+  if (in_dtype != WUSHKV_BF16 && in_dtype != WUSHKV_FP32) return WUSHKV_ERR_UNSUPPORTED;
+  if (n_new <= 0 || !k_new || !v_new || !start_pos || !data) return WUSHKV_ERR_INVALID;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(start_pos, 4) || !aligned(data, 16))
+    return WUSHKV_ERR_MISALIGNED;
+  if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
+  if (in_dtype != WUSHKV_BF16 || (int64_t)cache->batch * n_new > 64) return WUSHKV_ERR_UNSUPPORTED;
+  cudaError_t e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, data, kind,
+                                                       kind == WUSHKV_TRANSFORM_BLOCK_DIAG ? block : 0, nullptr, 0,
+                                                       status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 

@@ -32,7 +32,8 @@ struct SmallArgs {
   int num_kv_heads, total_rows, n_new, capacity;
   CacheRows rows;                   // (sequence, head, position) -> row, contiguous or paged
   const int32_t* start_pos;
-  const float* tk;                  // [Hkv][128][128] or nullptr
+  const float* tk;                  // dense [Hkv][128][128], blocks [Hkv][128/b][b][b], scales [Hkv][128], or nullptr
+  int tkind, tblock;                // transform variant (kTf*), block size of the block-diagonal one
   const float* rope;                // [rope_rows][128] (cos | sin per position) or nullptr
   int rope_rows;
   uint8_t* k_codes;
@@ -162,7 +163,14 @@ __device__ void quantize_group_warp(const float* x, const SmallArgs& a, bool sto
   }
 }
 
-template <int BITS, int KIND, bool TRANSFORM, bool ROPE>
+// Key transform variants: none (keys given transformed), dense T_k, block-diagonal T_k
+// (blocks of tblock x tblock on the diagonal), and T_k = H diag(s) / sqrt(128).
+enum { kTfNone = 0, kTfDense = 1, kTfBlock = 2, kTfHadamard = 3 };
+static_assert(kTfDense == WUSHKV_TRANSFORM_DENSE && kTfBlock == WUSHKV_TRANSFORM_BLOCK_DIAG &&
+                  kTfHadamard == WUSHKV_TRANSFORM_HADAMARD_DIAG,
+              "transform kinds follow the C ABI");
+
+template <int BITS, int KIND, int TF, bool ROPE>
 __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
   __shared__ __align__(16) float xk[kRows][kHeadDim];   // keys (transformed)
   __shared__ __align__(16) float xv[kRows][kHeadDim];   // values
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
     const size_t off = ((size_t)(f0 + r) * a.num_kv_heads + h) * kHeadDim + c;
     xv[r][c] = __bfloat162float(a.v[off]);
     const float kv = __bfloat162float(a.k[off]);
-    if (TRANSFORM || ROPE) kr[r][c] = kv;
+    if (TF != kTfNone || ROPE) kr[r][c] = kv;
     else xk[r][c] = kv;
   }
   __syncthreads();
@@ -195,13 +203,13 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
         rx = fmaf(x, cs, -(y * sn));
         ry = fmaf(y, cs, x * sn);
       }
-      float* dst = TRANSFORM ? kr[r] : xk[r];
+      float* dst = TF != kTfNone ? kr[r] : xk[r];
       dst[c] = rx;
       dst[c + kHeadDim / 2] = ry;
     }
     __syncthreads();
   }
-  if (TRANSFORM) {
+  if (TF == kTfDense) {
     // x[r][i] = sum_j T[i][j] k[r][j]: thread i reads row i of T once for every row r
     const float4* trow = reinterpret_cast<const float4*>(a.tk + ((size_t)h * kHeadDim + tid) * kHeadDim);
     float acc[kRows][4];
@@ -222,6 +230,51 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
       if (r < nrows) xk[r][tid] = (acc[r][0] + acc[r][1]) + (acc[r][2] + acc[r][3]);
+    __syncthreads();
+  }
+  if (TF == kTfBlock) {
+    // x[r][i] = sum_j B[i / b][i % b][j] k[r][(i / b) b + j]: the dense loop restricted to
+    // the block, in the same four chains (the dense product of the expanded matrix adds
+    // only exact zeros besides these terms)
+    const int bs = a.tblock, blk = tid / bs, ii = tid % bs;
+    const float4* brow =
+        reinterpret_cast<const float4*>(a.tk + (((size_t)h * (kHeadDim / bs) + blk) * bs + ii) * bs);
+    float acc[kRows][4];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
+    for (int j = 0; j < bs / 4; ++j) {
+      const float4 t = __ldg(brow + j);
+#pragma unroll
+      for (int r = 0; r < kRows; ++r) {
+        const float4 k4 = reinterpret_cast<const float4*>(kr[r] + blk * bs)[j];
+        acc[r][0] = fmaf(t.x, k4.x, acc[r][0]);
+        acc[r][1] = fmaf(t.y, k4.y, acc[r][1]);
+        acc[r][2] = fmaf(t.z, k4.z, acc[r][2]);
+        acc[r][3] = fmaf(t.w, k4.w, acc[r][3]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+      if (r < nrows) xk[r][tid] = (acc[r][0] + acc[r][1]) + (acc[r][2] + acc[r][3]);
+    __syncthreads();
+  }
+  if (TF == kTfHadamard) {
+    // x = H (s * k) / sqrt(128): scale, then the seven butterfly stages of the Sylvester
+    // Hadamard transform in place (stage `half` pairs channels base and base + half)
+    const float sc = __ldg(a.tk + (size_t)h * kHeadDim + tid);
+    for (int r = 0; r < nrows; ++r) kr[r][tid] *= sc;
+    __syncthreads();
+    for (int half = kHeadDim / 2; half >= 1; half >>= 1) {
+      for (int e = tid; e < nrows * (kHeadDim / 2); e += kThreads) {
+        const int r = e / (kHeadDim / 2), p = e % (kHeadDim / 2);
+        const int base = (p / half) * (2 * half) + p % half;
+        const float u = kr[r][base], v = kr[r][base + half];
+        kr[r][base] = u + v;
+        kr[r][base + half] = u - v;
+      }
+      __syncthreads();
+    }
+    for (int r = 0; r < nrows; ++r) xk[r][tid] = kr[r][tid] * 0.08838834764831845f;   // 1 / sqrt(128)
     __syncthreads();
   }
   const int warp = tid >> 5;
@@ -246,11 +299,22 @@ __global__ void __launch_bounds__(kThreads) append_small_kernel(SmallArgs a) {
 template <int BITS, int KIND>
 cudaError_t launch_kind(const SmallArgs& a, cudaStream_t stream) {
   dim3 grid(a.num_kv_heads, (a.total_rows + kRows - 1) / kRows);
-  const bool tf = a.tk != nullptr, rope = a.rope != nullptr;
-  if (tf && rope) append_small_kernel<BITS, KIND, true, true><<<grid, kThreads, 0, stream>>>(a);
-  else if (tf) append_small_kernel<BITS, KIND, true, false><<<grid, kThreads, 0, stream>>>(a);
-  else if (rope) append_small_kernel<BITS, KIND, false, true><<<grid, kThreads, 0, stream>>>(a);
-  else append_small_kernel<BITS, KIND, false, false><<<grid, kThreads, 0, stream>>>(a);
+  const bool rope = a.rope != nullptr;
+  switch (a.tk == nullptr ? (int)kTfNone : a.tkind) {
+    case kTfDense:
+      if (rope) append_small_kernel<BITS, KIND, kTfDense, true><<<grid, kThreads, 0, stream>>>(a);
+      else append_small_kernel<BITS, KIND, kTfDense, false><<<grid, kThreads, 0, stream>>>(a);
+      break;
+    case kTfBlock:
+      append_small_kernel<BITS, KIND, kTfBlock, false><<<grid, kThreads, 0, stream>>>(a);
+      break;
+    case kTfHadamard:
+      append_small_kernel<BITS, KIND, kTfHadamard, false><<<grid, kThreads, 0, stream>>>(a);
+      break;
+    default:
+      if (rope) append_small_kernel<BITS, KIND, kTfNone, true><<<grid, kThreads, 0, stream>>>(a);
+      else append_small_kernel<BITS, KIND, kTfNone, false><<<grid, kThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -266,8 +330,8 @@ cudaError_t launch_bits(const SmallArgs& a, int bits, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                         const int32_t* start_pos, const float* Tk, const float* rope,
-                                         int rope_rows, int32_t* status, cudaStream_t stream) {
+                                         const int32_t* start_pos, const float* Tk, int tkind, int tblock,
+                                         const float* rope, int rope_rows, int32_t* status, cudaStream_t stream) {
   SmallArgs a{};
   a.k = static_cast<const __nv_bfloat16*>(k_new);
   a.v = static_cast<const __nv_bfloat16*>(v_new);
@@ -278,6 +342,8 @@ cudaError_t launch_quantize_append_small(const wushkv_cache& c, const void* k_ne
   a.rows = CacheRows::of(c);
   a.start_pos = start_pos;
   a.tk = Tk;
+  a.tkind = tkind;
+  a.tblock = tblock;
   a.rope = rope;
   a.rope_rows = rope_rows;
   a.k_codes = c.k_codes;

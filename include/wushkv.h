@@ -163,6 +163,34 @@ WUSHKV_API int wushkv_quantize_append_rope(const wushkv_cache* cache, const void
                                 int32_t in_dtype, int32_t n_new, const int32_t* start_pos, const float* Tk,
                                 const float* rope_table, int32_t rope_rows, int32_t* status, void* stream);
 
+/* Key transform families ([ai4s 6]: cheaper structured transforms are the authors'
+ * future work; Hadamard is a baseline), all invertible T_k applied as x = T_k k:
+ *   DENSE         - data fp32 [Hkv][128][128] row-major (as Tk above);
+ *   BLOCK_DIAG    - data fp32 [Hkv][128/b][b][b]: block j (row-major) acts on channels
+ *                   [j b, (j+1) b), b = 16, 32 or 64;
+ *   HADAMARD_DIAG - data fp32 s [Hkv][128]: T_k = H diag(s) / sqrt(128), H the
+ *                   Sylvester Hadamard matrix (H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]);
+ *                   its query map is the same family with 1/s. */
+typedef enum {
+  WUSHKV_TRANSFORM_DENSE = 1,
+  WUSHKV_TRANSFORM_BLOCK_DIAG = 2,
+  WUSHKV_TRANSFORM_HADAMARD_DIAG = 3
+} wushkv_transform_kind;
+
+/* wushkv_quantize_append with a structured key transform: block-diagonal keys cost b
+ * instead of 128 multiply-adds per channel, Hadamard-diagonal ones a scale and a
+ * seven-stage butterfly.  kind is a wushkv_transform_kind; block is b for BLOCK_DIAG
+ * (ignored otherwise); data is device fp32, 16-byte aligned, laid out as above.
+ * DENSE takes every call wushkv_quantize_append takes.  The structured kinds are built
+ * for decode-step appends (bf16, batch * n_new <= 64 token rows); other calls return
+ * WUSHKV_ERR_UNSUPPORTED.  Results equal wushkv_quantize_append given the expanded
+ * dense T_k up to the fp32 rounding of the transform; for BLOCK_DIAG they are
+ * identical to the decode-step path given the expanded matrix.  Other arguments,
+ * errors and status bits as wushkv_quantize_append. */
+WUSHKV_API int wushkv_quantize_append_structured(const wushkv_cache* cache, const void* k_new, const void* v_new,
+                                      int32_t in_dtype, int32_t n_new, const int32_t* start_pos, int32_t kind,
+                                      int32_t block, const float* data, int32_t* status, void* stream);
+
 /* Decode-query map q' = T_k^{-T} q, with T_k of the query head's KV head h / g,
  * g = num_q_heads / num_kv_heads.  Needed because keys are cached as T_k k, and
  * (T_k^{-T} q) . (T_k k) = q . k keeps the attention scores unchanged (implied by

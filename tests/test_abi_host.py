@@ -226,3 +226,27 @@ def test_append_rope_argument_checks():
     assert call(dt=1) == _lib.ERR_UNSUPPORTED            # fp32 keys
     assert call(dt=7) == _lib.ERR_UNSUPPORTED
     assert call(n=0) == _lib.ERR_INVALID
+
+
+def test_append_structured_argument_checks():
+    lib = dq.library()
+    d = _desc()
+    f = lib.wushkv_quantize_append_structured
+    ok = (ctypes.byref(d), 0x50000, 0x60000, 0, 4, 0x70000, 2, 32, 0x80000, None, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["c", "k", "v", "dt", "n", "sp", "kind", "block", "data", "st", "stream"]
+        for key, val in kw.items():
+            args[names.index(key)] = val
+        return f(*args)
+
+    assert call(kind=9) == _lib.ERR_UNSUPPORTED
+    assert call(block=8) == _lib.ERR_UNSUPPORTED
+    assert call(block=128) == _lib.ERR_UNSUPPORTED
+    assert call(data=None) == _lib.ERR_INVALID
+    assert call(data=0x80004) == _lib.ERR_MISALIGNED
+    assert call(n=33) == _lib.ERR_UNSUPPORTED            # not a decode-step append
+    assert call(kind=3, dt=1) == _lib.ERR_UNSUPPORTED     # fp32 keys
+    assert call(kind=1, data=None) == _lib.ERR_INVALID    # dense needs its matrix
+    assert call(kind=1, dt=7) == _lib.ERR_UNSUPPORTED     # dense forwards to the plain append's checks
