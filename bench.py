@@ -373,6 +373,8 @@ def run_ours(args, rank, world, local):
     chunk = bench_chunk(dq, device, args, world)
     # decode-step append with RoPE fused in front of the transform
     rope_app = bench_rope_append(dq, device, args, world)
+    # decode-step append with structured key transforms
+    struct_app = bench_structured_append(dq, device, args, world)
     st = int(status.item())
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -393,6 +395,7 @@ def run_ours(args, rank, world, local):
         "paged_decode": paged,
         "chunk_attention": chunk,
         "append_rope": rope_app,
+        "append_structured": struct_app,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -532,6 +535,50 @@ def bench_rope_append(dq, device, args, world):
     plain = timed(lambda: dq.quantize_append(cache, k_post, v, sp, tk))
     return {"workload": f"{w.name}: 1 token x 16 sequences x 8 KV heads", "fused_rope_us": round(fused * 1e3, 2),
             "post_rope_input_us": round(plain * 1e3, 2), "calls": reps, "l2": "inputs L2-warm (back-to-back calls)"}
+
+
+def bench_structured_append(dq, device, args, world):
+    """Decode-step append (one token for each of 16 sequences x 8 KV heads, affine 2-bit)
+    with a dense, a block-diagonal (b = 32) and a Hadamard-diagonal key transform:
+    back-to-back calls between two events (inputs L2-warm).  A failure is reported in
+    the returned object, so that the main measurement line still prints."""
+    try:
+        w = QWEN8B_DECODE
+        qs = w.quant
+        cap = 4096
+        cache = dq.PackedCache(w.batch, w.num_kv_heads, cap, qs.kind, qs.bits, qs.clip_alpha, device=device)
+        sp = torch.arange(w.batch, dtype=torch.int32, device=device) * 200
+        k = gen.keys(w, 0, w.batch, sp.tolist(), 1, device=device)
+        v = gen.values(w, 0, w.batch, sp.tolist(), 1, device=device)
+        dense = torch.from_numpy(gen.transforms(w)[0]).to(device)
+        g = torch.Generator().manual_seed(5)
+        blocks = (torch.randn(w.num_kv_heads, 4, 32, 32, generator=g) / 32 ** 0.5).to(device)
+        scales = (torch.rand(w.num_kv_heads, 128, generator=g) * 3.75 + 0.25).to(device)
+        stream = torch.cuda.current_stream(device)
+        reps = max(50, 10 * args.steps)
+
+        def timed(fn):
+            for _ in range(max(3, args.warmup)):
+                fn()
+            torch.cuda.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            return max_over_ranks(a.elapsed_time(b) / reps, world)
+
+        t_dense = timed(lambda: dq.quantize_append(cache, k, v, sp, dense))
+        t_block = timed(lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_BLOCK_DIAG, blocks,
+                                                              block=32))
+        t_had = timed(lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_HADAMARD_DIAG, scales))
+        return {"workload": f"{w.name}: 1 token x 16 sequences x 8 KV heads", "dense_us": round(t_dense * 1e3, 2),
+                "block_diag_32_us": round(t_block * 1e3, 2), "hadamard_diag_us": round(t_had * 1e3, 2),
+                "calls": reps, "l2": "inputs L2-warm (back-to-back calls)"}
+    except Exception as e:  # noqa: BLE001 - reported in the output line
+        return {"error": f"{type(e).__name__}: {e}"}
 
 
 def bench_append(dq, device, args, world):
