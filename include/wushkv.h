@@ -22,7 +22,8 @@
  *     on the device (see WUSHKV_STATUS_*) are OR-ed into the optional `status`
  *     int32 (device memory, caller clears it); no kernel ever traps.
  *   - Calls keep no state between them and are safe to issue from several
- *     host threads on different streams.
+ *     host threads on different streams (except wushkv_decode_attention_noalloc,
+ *     whose fixed scratch array is shared; see its declaration).
  */
 #ifndef WUSHKV_H_
 #define WUSHKV_H_
