@@ -196,7 +196,7 @@ int wushkv_chunk_attention(const wushkv_cache* cache, const float* q_t, int32_t 
 size_t wushkv_decode_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads, int32_t num_splits) {
   if (check_cache(cache, false) != WUSHKV_OK) return 0;
   if (check_heads(num_q_heads, cache->num_kv_heads) != WUSHKV_OK) return 0;
-  if (num_splits < 0) return 0;
+  if (num_splits < 0 || num_splits > 4096) return 0;
   return wushkv::decode_workspace_bytes(*cache, num_q_heads, num_splits);
 }
 

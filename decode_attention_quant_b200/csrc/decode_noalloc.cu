@@ -12,7 +12,13 @@
 // kernel writes every partial (m, l, o) of every split before the combine kernel
 // reads it.  Two calls that may run at the same time on one device (different
 // streams, or different host threads without ordering) race on the array.
-#include <atomic>
+//
+// The array's device address belongs to the CUDA context that loaded this module.
+// It is looked up once per context (the first call after a context is made current
+// on a device, e.g. the first call on that device, or the first after the primary
+// context was reset by cudaDeviceReset) and cached with the context handle.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "wushkv_launch.h"
@@ -23,27 +29,56 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_decode_scratch[WUSHKV_DECODE_STATIC_SCRATCH_BYTES];
 
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
+struct ScratchSlot {
+  CUcontext ctx;   // context the address was looked up in
+  void* ptr;       // device address of g_decode_scratch in that context
+};
+ScratchSlot g_slots[kMaxDevices];
 std::mutex g_setup_mutex;
 
-// Device address of g_decode_scratch on the current device, looked up once per device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of g_decode_scratch in the current device's current context.
 int scratch_on_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return wushkv::record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return WUSHKV_ERR_UNSUPPORTED;
-  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      e = cudaGetSymbolAddress(&p, g_decode_scratch);
-      if (e == cudaSuccess && p == nullptr) e = cudaErrorInvalidSymbol;
-      if (e != cudaSuccess) return wushkv::record_cuda_error(e);
-      g_scratch_ptr[dev].store(p, std::memory_order_release);
-    }
+  CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return wushkv::record_cuda_error(cudaErrorNotSupported);
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return wushkv::record_cuda_error(cudaErrorDeviceUninitialized);
+  if (ctx == nullptr) {
+    // no context current on this thread yet: make the device's primary context current
+    // (the one the kernels below run in), then read its handle
+    e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return wushkv::record_cuda_error(e);
+    if (get(&ctx) != CUDA_SUCCESS || ctx == nullptr) return wushkv::record_cuda_error(cudaErrorDeviceUninitialized);
   }
-  *out = p;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  ScratchSlot& s = g_slots[dev];
+  if (s.ptr == nullptr || s.ctx != ctx) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e == cudaSuccess && p == nullptr) e = cudaErrorInvalidSymbol;
+    if (e != cudaSuccess) return wushkv::record_cuda_error(e);
+    s.ctx = ctx;
+    s.ptr = p;
+  }
+  *out = s.ptr;
   return WUSHKV_OK;
 }
 

@@ -14,7 +14,7 @@
 //           with p_t scale_t rounded to 16-bit integers pi = u0 + 2^8 u1 (per tile and
 //           head, F = the tile's largest p_t scale_t) split into two uint8 limbs.
 // (QuEST: scale = Delta, zero = -(2^(b-1) - 1/2) Delta.)  The softmax is online in the
-// log2 domain across 128-token tiles.
+// log2 domain across 256-token tiles.
 //
 // One CTA = one (sequence, KV head, split); tiles of 256 tokens, five warps:
 //   warp 0      one thread: TMA copies of each tile's packed K and V codes into a

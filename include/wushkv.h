@@ -204,8 +204,9 @@ WUSHKV_API int wushkv_transform_query(const void* q, int32_t q_dtype, int32_t ba
                            int32_t num_kv_heads, const float* Tk_invT, float* q_out, void* stream);
 
 /* Bytes of decode workspace needed for wushkv_decode_attention with the same
- * cache shape, num_q_heads and num_splits (0 = the automatic split count).
- * Returns 0 for invalid arguments.  Host only; no CUDA call. */
+ * cache shape, num_q_heads and num_splits (0 = the automatic split count, else
+ * 1 .. 4096).  Returns 0 for invalid arguments.  Host only: it enqueues nothing (the
+ * automatic split count reads the current device's SM count). */
 WUSHKV_API size_t wushkv_decode_workspace_bytes(const wushkv_cache* cache, int32_t num_q_heads,
                                      int32_t num_splits);
 
@@ -242,9 +243,12 @@ WUSHKV_API int wushkv_decode_attention(const wushkv_cache* cache, const float* q
  *   - WUSHKV_ERR_WORKSPACE when wushkv_decode_workspace_bytes(cache, num_q_heads,
  *     num_splits) exceeds WUSHKV_DECODE_STATIC_SCRATCH_BYTES (pass a smaller
  *     num_splits, or use wushkv_decode_attention with a workspace);
- *   - the first call on each device looks up the array's device address on the
- *     current device (a CUDA runtime call, no allocation by this library); make that
- *     first call before any stream capture on that device;
+ *   - the first call on each device looks up the array's device address in the
+ *     device's current CUDA context (a CUDA runtime call, no allocation by this
+ *     library) and keeps it for later calls in that context; a call in a new context
+ *     on the device (for instance after cudaDeviceReset) looks it up again.  Make the
+ *     first call on a device, and the first after a reset, before any stream capture
+ *     on that device;
  *   - every call on a device shares the one array and leaves its partials there;
  *     nothing in it needs clearing between calls (each call writes every partial it
  *     reads), but calls that may overlap in time on one device (different streams,

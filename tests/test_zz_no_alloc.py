@@ -41,6 +41,11 @@ def test_rejects_oversized_and_invalid_without_launching():
                                                1, vp(0), vp(0)) == _lib.ERR_UNSUPPORTED
     assert lib.wushkv_decode_attention_noalloc(ctypes.byref(d), vp(0x50000), 32, vp(0x60000), TAU, vp(0x70000),
                                                -1, vp(0), vp(0)) == _lib.ERR_INVALID
+    # a split count out of range is invalid whatever the scratch it would need
+    d = _fake_desc(2048, 8, 256)
+    assert lib.wushkv_decode_workspace_bytes(ctypes.byref(d), 32, 5000) == 0
+    assert lib.wushkv_decode_attention_noalloc(ctypes.byref(d), vp(0x50000), 32, vp(0x60000), TAU, vp(0x70000),
+                                               5000, vp(0), vp(0)) == _lib.ERR_INVALID
 
 
 @pytest.mark.gpu
