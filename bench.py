@@ -32,7 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from synth import gen  # noqa: E402
-from synth.configs import QWEN8B_DECODE, QWEN8B_SWEEP, quest  # noqa: E402
+from synth.configs import QWEN8B_DECODE, QWEN8B_LONG, QWEN8B_SWEEP, QWEN32B_STACK, quest  # noqa: E402
 
 METRIC = "2-bit KV decode-attn HBM GB/s (% of peak) & quant-append tokens/s, 1×B200"
 TAU = 1.0 / math.sqrt(128)
@@ -375,6 +375,11 @@ def run_ours(args, rank, world, local):
     rope_app = bench_rope_append(dq, device, args, world)
     # decode-step append with structured key transforms
     struct_app = bench_structured_append(dq, device, args, world)
+    # every workload's decode call and the sweep's chunk appends at 3 and 4 bits
+    dec_all = bench_decode_workloads(dq, device, args, world)
+    app_all = [app] + [bench_append(dq, device, args, world, bits=b) for b in (3, 4)]
+    # the 64-layer Qwen3-32B-shaped stack, one CUDA graph per step
+    stack = bench_stack(dq, device, args, world)
     st = int(status.item())
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -396,6 +401,9 @@ def run_ours(args, rank, world, local):
         "chunk_attention": chunk,
         "append_rope": rope_app,
         "append_structured": struct_app,
+        "decode_workloads": dec_all,
+        "append_workloads": app_all,
+        "stack": stack,
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -581,8 +589,118 @@ def bench_structured_append(dq, device, args, world):
         return {"error": f"{type(e).__name__}: {e}"}
 
 
-def bench_append(dq, device, args, world):
-    w = QWEN8B_SWEEP(2)
+def bench_decode_workloads(dq, device, args, world):
+    """One decode call on each workload shape (random packed caches of the full context,
+    all larger than L2): K back-to-back calls between two events.  Bytes: the cache's
+    codes and meta of K and V up to ctx, plus q' in and the output out."""
+    peak, _ = _peaks()
+    res = []
+    for w in (QWEN8B_DECODE, QWEN8B_SWEEP(2), QWEN8B_SWEEP(3), QWEN8B_SWEEP(4), QWEN8B_LONG, QWEN32B_STACK):
+        try:
+            qs = w.quant
+            c = gen.random_cache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, seed=w.seed, device=device)
+            cache = dq.PackedCache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, qs.clip_alpha, qs.rank_lo,
+                                   qs.rank_hi, tensors=c)
+            q = torch.randn(w.batch, w.num_q_heads, 128, generator=torch.Generator(device=device).manual_seed(2),
+                            device=device)
+            ctx = torch.full((w.batch,), w.ctx, dtype=torch.int32, device=device)
+            out = torch.empty_like(q)
+            ws = torch.empty(dq.decode_workspace_bytes(cache, w.num_q_heads), dtype=torch.uint8, device=device)
+            stream = torch.cuda.current_stream(device)
+            for _ in range(max(3, args.warmup)):
+                dq.decode_attention(cache, q, ctx, TAU, out=out, workspace=ws)
+            torch.cuda.synchronize()
+            reps = max(5, args.steps)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                dq.decode_attention(cache, q, ctx, TAU, out=out, workspace=ws)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = max_over_ranks(a.elapsed_time(b) / reps, world)
+            by = decode_bytes(w, [w.ctx] * w.batch)
+            gbs = by / (ms * 1e-3) / 1e9
+            res.append({"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "ctx": w.ctx,
+                        "bits": qs.bits, "quantizer": "quest" if qs.kind == 0 else "affine", "ms": round(ms, 5),
+                        "GB/s": round(world * gbs, 1), "frac_of_peak": round(gbs / peak, 4), "alg_bytes": by,
+                        "tokens_per_s": round(world * w.batch * w.ctx / (ms * 1e-3), 1),
+                        "splits": int(dq.decode_workspace_bytes(cache, w.num_q_heads)
+                                      // (w.batch * w.num_q_heads * 132 * 4)),
+                        "l2": "cache larger than L2, back-to-back calls"})
+            del c, cache, q, out, ws
+        except Exception as e:  # noqa: BLE001 - reported in the output line
+            res.append({"workload": w.name, "error": f"{type(e).__name__}: {e}"})
+    return res
+
+
+def bench_stack(dq, device, args, world):
+    """The Qwen3-32B-shaped 64-layer stack: per layer the append of a 16-token chunk per
+    sequence (QuEST 2-bit, own T_k), the query map and decode attention at context 8192,
+    all 64 layers captured in one CUDA graph; K replays between two events.  The caches'
+    history is random packed data (the kernels' time does not depend on the values)."""
+    try:
+        w = QWEN32B_STACK
+        qs = w.quant
+        n = w.append_tokens
+        start = torch.full((w.batch,), w.history, dtype=torch.int32, device=device)
+        ctx = torch.full((w.batch,), w.ctx, dtype=torch.int32, device=device)
+        status = torch.zeros(1, dtype=torch.int32, device=device)
+        layers = []
+        for layer in range(w.layers):
+            tk, tinv = gen.transforms(w, layer)
+            c = gen.random_cache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, seed=w.seed + layer, device=device)
+            cache = dq.PackedCache(w.batch, w.num_kv_heads, w.ctx, qs.kind, qs.bits, qs.clip_alpha, tensors=c)
+            q = gen.queries(w, layer, device=device).contiguous()
+            layers.append((cache, gen.keys(w, 0, w.batch, w.history, n, layer=layer, device=device, salt=1),
+                           gen.values(w, 0, w.batch, w.history, n, layer=layer, device=device, salt=1),
+                           torch.from_numpy(tk).to(device), torch.from_numpy(tinv).to(device), q,
+                           torch.empty(q.shape, dtype=torch.float32, device=device),
+                           torch.empty(q.shape, dtype=torch.float32, device=device),
+                           torch.empty(dq.decode_workspace_bytes(cache, w.num_q_heads), dtype=torch.uint8,
+                                       device=device)))
+
+        def step():
+            for cache, k, v, tk, tinv, q, q_t, out, ws in layers:
+                dq.quantize_append(cache, k, v, start, tk, status)
+                dq.transform_query(q, tinv, w.num_kv_heads, out=q_t)
+                dq.decode_attention(cache, q_t, ctx, TAU, out=out, workspace=ws, status=status)
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream(device)
+        reps = max(3, min(args.steps, 10))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(a.elapsed_time(b) / reps, world)
+        del graph
+        dec = w.layers * decode_bytes(w, [w.ctx] * w.batch)
+        by = dec + w.layers * (append_bytes(w, n) + query_bytes(w))
+        peak, _ = _peaks()
+        return {"workload": f"{w.name}: per layer 16-token append + query map + decode, 64 layers",
+                "ms_per_step": round(ms, 4), "step_bytes": by, "decode_bytes": dec,
+                "GB/s": round(world * by / (ms * 1e-3) / 1e9, 1), "frac_of_peak": round(by / (ms * 1e-3) / 1e9 / peak, 4),
+                "launches_per_step": w.layers * (APPEND_LAUNCHES + QUERY_LAUNCHES + DECODE_LAUNCHES),
+                "ms_at_70pct_of_peak": round(by / (0.7 * peak * 1e9) * 1e3, 4), "replays": reps,
+                "device_status": int(status.item()), "launch": "one CUDA graph per step",
+                "l2": "caches larger than L2 (142.6 MB per layer)"}
+    except Exception as e:  # noqa: BLE001 - reported in the output line
+        return {"error": f"{type(e).__name__}: {e}"}
+
+
+def bench_append(dq, device, args, world, bits=2):
+    w = QWEN8B_SWEEP(bits)
     qs = w.quant
     tk = torch.from_numpy(gen.transforms(w)[0]).to(device)
     n = w.append_tokens

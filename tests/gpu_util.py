@@ -99,3 +99,49 @@ def check_key_rows(oc, gc, x, kind, bits, start, alpha):
         code_diffs += int(off.sum())
         near += int((dist <= 1e-4 * step).sum())
     return meta_flips, code_diffs, near
+
+
+def append_history(cache, w, n_tokens, tk, layer=0, chunk=4096):
+    """Fill positions 0 .. n_tokens-1 of every sequence with the GPU's own appends of the
+    workload's synthetic keys and values (chunks of `chunk` tokens; tk a device tensor)."""
+    t = 0
+    status = torch.zeros(1, dtype=torch.int32, device=cache.device)
+    while t < n_tokens:
+        n = min(chunk, n_tokens - t)
+        k = gen_keys(w, t, n, layer, cache.device)
+        v = gen_values(w, t, n, layer, cache.device)
+        sp = torch.full((w.batch,), t, dtype=torch.int32, device=cache.device)
+        dq.quantize_append(cache, k, v, sp, tk, status)
+        t += n
+    torch.cuda.synchronize()
+    return int(status.item())
+
+
+def gen_keys(w, t0, n, layer, device):
+    from synth import gen
+    return gen.keys(w, 0, w.batch, t0, n, layer=layer, device=device)
+
+
+def gen_values(w, t0, n, layer, device):
+    from synth import gen
+    return gen.values(w, 0, w.batch, t0, n, layer=layer, device=device)
+
+
+def decode_vs_oracle(cache_np, q_t, ctx, tau, kind, bits, num_kv_heads, out, pairs=None):
+    """Oracle decode (fp64) of the (sequence, KV head) pairs listed (all when None) over the
+    given numpy cache, against the GPU output `out` [B, Hq, 128]; returns the worst
+    (max-abs, rel-L2) over the pairs and the number of pairs checked."""
+    import oracle.wushkv_oracle as orc_
+    bsz, hq, _ = q_t.shape
+    g = hq // num_kv_heads
+    if pairs is None:
+        pairs = [(b, kv) for b in range(bsz) for kv in range(num_kv_heads)]
+    worst_ma = worst_rl = 0.0
+    for (b, kv) in pairs:
+        n = int(min(ctx[b], cache_np["k_codes"].shape[2]))
+        ref = orc_.decode_attention_pair(cache_np["k_codes"][b, kv, :n], cache_np["k_meta"][b, kv, :n],
+                                         cache_np["v_codes"][b, kv, :n], cache_np["v_meta"][b, kv, :n],
+                                         q_t[b, kv * g:(kv + 1) * g], tau, kind, bits)
+        ma, rl = attention_errors(out[b, kv * g:(kv + 1) * g], ref)
+        worst_ma, worst_rl = max(worst_ma, ma), max(worst_rl, rl)
+    return worst_ma, worst_rl, len(pairs)
