@@ -509,6 +509,30 @@ def bench_chunk(dq, device, args, world):
     return res
 
 
+def device_time_per_call(fn, reps, args, world):
+    """Device time (ms) per call of `fn`: `reps` calls captured back to back in one CUDA
+    graph and replayed between two events, so that the host's per-call work (argument
+    checks, marshalling) cannot leave the device idle between short launches."""
+    for _ in range(max(3, args.warmup)):
+        fn()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(reps):
+            fn()
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    return max_over_ranks(a.elapsed_time(b) / reps, world)
+
+
 def bench_rope_append(dq, device, args, world):
     """Decode-step append (one token for each of 16 sequences x 8 KV heads, Qwen3-8B
     shapes, affine 2-bit) with RoPE fused in front of the transform, against the same
@@ -523,26 +547,13 @@ def bench_rope_append(dq, device, args, world):
     k_pre = gen.keys(w, 0, w.batch, sp.tolist(), 1, rope=False, device=device)
     k_post = gen.keys(w, 0, w.batch, sp.tolist(), 1, device=device)
     v = gen.values(w, 0, w.batch, sp.tolist(), 1, device=device)
-    stream = torch.cuda.current_stream(device)
     reps = max(50, 10 * args.steps)
-
-    def timed(fn):
-        for _ in range(max(3, args.warmup)):
-            fn()
-        torch.cuda.synchronize()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b) / reps, world)
-
-    fused = timed(lambda: dq.quantize_append_rope(cache, k_pre, v, sp, table, tk))
-    plain = timed(lambda: dq.quantize_append(cache, k_post, v, sp, tk))
+    fused = device_time_per_call(lambda: dq.quantize_append_rope(cache, k_pre, v, sp, table, tk), reps, args, world)
+    plain = device_time_per_call(lambda: dq.quantize_append(cache, k_post, v, sp, tk), reps, args, world)
     return {"workload": f"{w.name}: 1 token x 16 sequences x 8 KV heads", "fused_rope_us": round(fused * 1e3, 2),
-            "post_rope_input_us": round(plain * 1e3, 2), "calls": reps, "l2": "inputs L2-warm (back-to-back calls)"}
+            "post_rope_input_us": round(plain * 1e3, 2), "calls": reps,
+            "timing": "device time of the calls captured back to back in one CUDA graph",
+            "l2": "inputs L2-warm (back-to-back calls)"}
 
 
 def bench_structured_append(dq, device, args, world):
@@ -562,29 +573,18 @@ def bench_structured_append(dq, device, args, world):
         g = torch.Generator().manual_seed(5)
         blocks = (torch.randn(w.num_kv_heads, 4, 32, 32, generator=g) / 32 ** 0.5).to(device)
         scales = (torch.rand(w.num_kv_heads, 128, generator=g) * 3.75 + 0.25).to(device)
-        stream = torch.cuda.current_stream(device)
         reps = max(50, 10 * args.steps)
-
-        def timed(fn):
-            for _ in range(max(3, args.warmup)):
-                fn()
-            torch.cuda.synchronize()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                fn()
-            b.record(stream)
-            torch.cuda.synchronize()
-            return max_over_ranks(a.elapsed_time(b) / reps, world)
-
-        t_dense = timed(lambda: dq.quantize_append(cache, k, v, sp, dense))
-        t_block = timed(lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_BLOCK_DIAG, blocks,
-                                                              block=32))
-        t_had = timed(lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_HADAMARD_DIAG, scales))
+        t_dense = device_time_per_call(lambda: dq.quantize_append(cache, k, v, sp, dense), reps, args, world)
+        t_block = device_time_per_call(
+            lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_BLOCK_DIAG, blocks, block=32),
+            reps, args, world)
+        t_had = device_time_per_call(
+            lambda: dq.quantize_append_structured(cache, k, v, sp, dq.TRANSFORM_HADAMARD_DIAG, scales),
+            reps, args, world)
         return {"workload": f"{w.name}: 1 token x 16 sequences x 8 KV heads", "dense_us": round(t_dense * 1e3, 2),
                 "block_diag_32_us": round(t_block * 1e3, 2), "hadamard_diag_us": round(t_had * 1e3, 2),
-                "calls": reps, "l2": "inputs L2-warm (back-to-back calls)"}
+                "calls": reps, "timing": "device time of the calls captured back to back in one CUDA graph",
+                "l2": "inputs L2-warm (back-to-back calls)"}
     except Exception as e:  # noqa: BLE001 - reported in the output line
         return {"error": f"{type(e).__name__}: {e}"}
 

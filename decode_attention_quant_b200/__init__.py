@@ -22,7 +22,8 @@ from ._lib import (BF16, FP32, PCT_AFFINE, QUEST_INT, STATUS_BAD_PAGE, STATUS_CA
 
 HEAD_DIM = 128
 
-__all__ = ["PackedCache", "quantize_append", "quantize_append_rope", "quantize_append_structured", "transform_query", "decode_attention",
+__all__ = ["PackedCache", "quantize_append", "quantize_append_rope", "quantize_append_structured", "transform_query",
+           "transform_query_structured", "decode_attention",
            "decode_attention_noalloc", "decode_workspace_bytes", "chunk_attention", "chunk_workspace_bytes",
            "QUEST_INT", "PCT_AFFINE", "WushkvError", "library"]
 
@@ -166,8 +167,9 @@ def quantize_append_structured(cache: PackedCache, k_new, v_new, start_pos, kind
                                stream=None):
     """quantize_append with a structured key transform (kind = TRANSFORM_BLOCK_DIAG with
     data fp32 [Hkv, 128/block, block, block], or TRANSFORM_HADAMARD_DIAG with data = s fp32
-    [Hkv, 128], T_k = H diag(s) / sqrt(128)); decode-step appends only (bf16, B * n_new <= 64).
-    TRANSFORM_DENSE takes data as the dense T_k of quantize_append."""
+    [Hkv, 128], T_k = H diag(s) / sqrt(128)); bf16 inputs (decode-step appends on the CUDA
+    cores, larger ones on the tensor cores).  TRANSFORM_DENSE takes data as the dense T_k of
+    quantize_append."""
     if k_new.shape != v_new.shape or k_new.dtype != v_new.dtype:
         raise ValueError("k_new and v_new must have the same shape and dtype")
     if k_new.dim() != 4 or k_new.shape[0] != cache.batch or k_new.shape[2] != cache.num_kv_heads \
@@ -203,6 +205,29 @@ def transform_query(q, tk_inv_t, num_kv_heads, out=None, stream=None):
     rc = library().wushkv_transform_query(_ptr(q), _dtype_code(q), q.shape[0], q.shape[1], int(num_kv_heads),
                                           _ptr(tk_inv_t), _ptr(out), _stream(q.device, stream))
     _lib.check(rc, "wushkv_transform_query")
+    return out
+
+
+def transform_query_structured(q, kind, data, num_kv_heads, block=0, out=None, stream=None):
+    """q' = T_k^{-T} q for a structured key transform: kind = TRANSFORM_BLOCK_DIAG with data
+    = the blocks of T_k^{-T} (fp32 [Hkv, 128/block, block, block]), TRANSFORM_HADAMARD_DIAG
+    with data = the key transform's scales s (fp32 [Hkv, 128]), or TRANSFORM_DENSE with
+    data = T_k^{-T} (fp32 [Hkv, 128, 128])."""
+    if q.dim() != 3 or q.shape[2] != HEAD_DIM or not q.is_contiguous():
+        raise ValueError("q must be contiguous [B, Hq, 128]")
+    shapes = {_lib.TRANSFORM_DENSE: (num_kv_heads, HEAD_DIM, HEAD_DIM),
+              _lib.TRANSFORM_BLOCK_DIAG: (num_kv_heads, HEAD_DIM // max(int(block), 1), int(block), int(block)),
+              _lib.TRANSFORM_HADAMARD_DIAG: (num_kv_heads, HEAD_DIM)}
+    if int(kind) not in shapes:
+        raise ValueError("unknown transform kind")
+    if data.dtype != torch.float32 or tuple(data.shape) != shapes[int(kind)] or not data.is_contiguous():
+        raise ValueError(f"transform data must be contiguous float32 {shapes[int(kind)]}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    rc = library().wushkv_transform_query_structured(_ptr(q), _dtype_code(q), q.shape[0], q.shape[1],
+                                                     int(num_kv_heads), int(kind), int(block), _ptr(data),
+                                                     _ptr(out), _stream(q.device, stream))
+    _lib.check(rc, "wushkv_transform_query_structured")
     return out
 
 

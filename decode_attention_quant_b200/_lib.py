@@ -40,6 +40,7 @@ EXPORTS = (
     "wushkv_quantize_append_rope",
     "wushkv_quantize_append_structured",
     "wushkv_transform_query",
+    "wushkv_transform_query_structured",
     "wushkv_decode_workspace_bytes",
     "wushkv_decode_attention",
     "wushkv_decode_attention_noalloc",
@@ -91,6 +92,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.wushkv_quantize_append_structured.restype = ctypes.c_int
     lib.wushkv_transform_query.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
     lib.wushkv_transform_query.restype = ctypes.c_int
+    lib.wushkv_transform_query_structured.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    lib.wushkv_transform_query_structured.restype = ctypes.c_int
     lib.wushkv_decode_workspace_bytes.argtypes = [cp, i32, i32]
     lib.wushkv_decode_workspace_bytes.restype = sz
     lib.wushkv_decode_attention.argtypes = [cp, vp, i32, vp, ctypes.c_float, vp, vp, sz, i32, vp, vp]

@@ -10,8 +10,8 @@
 
 namespace wushkv {
 cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                      const int32_t* start_pos, const float* Tk, int32_t* status,
-                                      cudaStream_t stream);
+                                      const int32_t* start_pos, const float* Tk, int tkind, int tblock,
+                                      int32_t* status, cudaStream_t stream);
 cudaError_t launch_quantize_append_simt(const wushkv_cache& c, const void* k_new, const void* v_new,
                                         int in_dtype, int n_new, const int32_t* start_pos,
                                         const float* Tk, int32_t* status, cudaStream_t stream);
@@ -101,7 +101,8 @@ int wushkv_quantize_append(const wushkv_cache* cache, const void* k_new, const v
     e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, Tk, WUSHKV_TRANSFORM_DENSE, 0,
                                              nullptr, 0, status, st);
   else if (in_dtype == WUSHKV_BF16)
-    e = wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, status, st);
+    e = wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, Tk, WUSHKV_TRANSFORM_DENSE, 0,
+                                          status, st);
   else
     e = wushkv::launch_quantize_append_simt(*cache, k_new, v_new, in_dtype, n_new, start_pos, Tk, status, st);
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
@@ -143,10 +144,35 @@ int wushkv_quantize_append_structured(const wushkv_cache* cache, const void* k_n
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(start_pos, 4) || !aligned(data, 16))
     return WUSHKV_ERR_MISALIGNED;
   if (status != nullptr && !aligned(status, 4)) return WUSHKV_ERR_MISALIGNED;
-  if (in_dtype != WUSHKV_BF16 || (int64_t)cache->batch * n_new > 64) return WUSHKV_ERR_UNSUPPORTED;
-  cudaError_t e = wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, data, kind,
-                                                       kind == WUSHKV_TRANSFORM_BLOCK_DIAG ? block : 0, nullptr, 0,
-                                                       status, static_cast<cudaStream_t>(stream));
+  if (in_dtype != WUSHKV_BF16) return WUSHKV_ERR_UNSUPPORTED;
+  if ((int64_t)cache->batch * n_new > (int64_t)1 << 30) return WUSHKV_ERR_INVALID;
+  const int tblock = kind == WUSHKV_TRANSFORM_BLOCK_DIAG ? block : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = (int64_t)cache->batch * n_new <= 64
+                      ? wushkv::launch_quantize_append_small(*cache, k_new, v_new, n_new, start_pos, data, kind,
+                                                             tblock, nullptr, 0, status, st)
+                      : wushkv::launch_quantize_append_tc(*cache, k_new, v_new, n_new, start_pos, data, kind, tblock,
+                                                          status, st);
+  return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
+}
+
+int wushkv_transform_query_structured(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t kind, int32_t block, const float* data,
+                                      float* q_out, void* stream) {
+  if (kind == WUSHKV_TRANSFORM_DENSE)
+    return wushkv_transform_query(q, q_dtype, batch, num_q_heads, num_kv_heads, data, q_out, stream);
+  if (kind != WUSHKV_TRANSFORM_BLOCK_DIAG && kind != WUSHKV_TRANSFORM_HADAMARD_DIAG) return WUSHKV_ERR_UNSUPPORTED;
+  if (kind == WUSHKV_TRANSFORM_BLOCK_DIAG && block != 16 && block != 32 && block != 64) return WUSHKV_ERR_UNSUPPORTED;
+  if (q_dtype != WUSHKV_BF16 && q_dtype != WUSHKV_FP32) return WUSHKV_ERR_UNSUPPORTED;
+  int rc = check_heads(num_q_heads, num_kv_heads);
+  if (rc != WUSHKV_OK) return rc;
+  if (batch <= 0 || !q || !data || !q_out) return WUSHKV_ERR_INVALID;
+  if (batch > 65535) return WUSHKV_ERR_INVALID;
+  if ((const void*)q == (const void*)q_out) return WUSHKV_ERR_INVALID;
+  if (!aligned(q, 16) || !aligned(data, 16) || !aligned(q_out, 16)) return WUSHKV_ERR_MISALIGNED;
+  cudaError_t e = wushkv::launch_transform_query_structured(q, q_dtype, batch, num_q_heads, num_kv_heads, kind,
+                                                            kind == WUSHKV_TRANSFORM_BLOCK_DIAG ? block : 0, data,
+                                                            q_out, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? WUSHKV_OK : cuda_fail(e);
 }
 

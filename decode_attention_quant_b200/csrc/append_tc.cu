@@ -51,7 +51,8 @@ struct TcArgs {
   CacheRows rows;          // (sequence, head, position) -> row, contiguous or paged
   int tiles_per_head, ctas_per_head;
   const int32_t* start_pos;
-  const float* tk;
+  const float* tk;          // dense [Hkv][128][128], blocks [Hkv][128/b][b][b] or scales [Hkv][128]
+  int tkind, tblock;        // wushkv_transform_kind of tk, block size b of the block-diagonal kind
   uint8_t* k_codes;
   uint8_t* v_codes;
   uint16_t* k_meta;
@@ -137,19 +138,37 @@ __device__ __forceinline__ void quantize_store(Loader& ld, const TcArgs& a, int 
   if (flags && f >= 0) report(a.status, flags);
 }
 
+// Entries T[i][j .. j+3] of KV head h's key transform as fp32: the dense matrix, the
+// expanded block-diagonal one (zero off the diagonal blocks) or H diag(s) / sqrt(128)
+// (H_ij = (-1)^popcount(i & j), the Sylvester Hadamard matrix).
+__device__ __forceinline__ float4 transform_entries(const TcArgs& a, int h, int i, int j) {
+  if (a.tkind == WUSHKV_TRANSFORM_BLOCK_DIAG) {
+    const int bs = a.tblock, blk = i / bs;
+    if (j / bs != blk) return make_float4(0.f, 0.f, 0.f, 0.f);   // b >= 16: j .. j+3 share a block
+    return __ldg(reinterpret_cast<const float4*>(
+        a.tk + (((size_t)h * (kHeadDim / bs) + blk) * bs + i % bs) * bs + j % bs));
+  }
+  if (a.tkind == WUSHKV_TRANSFORM_HADAMARD_DIAG) {
+    const float4 sv = __ldg(reinterpret_cast<const float4*>(a.tk + (size_t)h * kHeadDim + j));
+    const float c = 0.08838834764831845f;                           // 1 / sqrt(128)
+    auto sgn = [&](int jj, float x) { return (__popc(i & jj) & 1) ? -(x * c) : x * c; };
+    return make_float4(sgn(j, sv.x), sgn(j + 1, sv.y), sgn(j + 2, sv.z), sgn(j + 3, sv.w));
+  }
+  return __ldg(reinterpret_cast<const float4*>(a.tk + ((size_t)h * kHeadDim + i) * kHeadDim + j));
+}
+
 // T_k[h] (fp32, row-major [i][j]) -> three bf16 planes, each laid out as the MMA's B
 // operand: K-major (j contiguous), two 64-column halves of 128 rows x 128 B, 16-byte
 // chunks swizzled by (row & 7).  P1 = bf16(T), P2 = bf16(T - P1), P3 = T - P1 - P2
 // (exact: the remainders of a 24-bit significand split into 8 + 8 + 8 bits).
-__device__ __forceinline__ void split_transform(const float* __restrict__ tk, uint8_t* planes, int tid,
-                                                int nthreads) {
+__device__ __forceinline__ void split_transform(const TcArgs& a, int h, uint8_t* planes, int tid, int nthreads) {
   // all of this thread's loads first (independent, so their latencies overlap)
   constexpr int kMaxPer = kHeadDim * kHeadDim / 4 / (kThreads - 64);
   float4 t4[kMaxPer];
 #pragma unroll
   for (int k = 0; k < kMaxPer; ++k) {
     const int q = tid + k * nthreads;
-    if (q < kHeadDim * kHeadDim / 4) t4[k] = __ldg(reinterpret_cast<const float4*>(tk) + q);
+    if (q < kHeadDim * kHeadDim / 4) t4[k] = transform_entries(a, h, q >> 5, (q & 31) * 4);
   }
 #pragma unroll
   for (int k = 0; k < kMaxPer; ++k) {
@@ -229,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_relinquish();
     }
     if (warp >= 2) {
-      split_transform(a.tk + (size_t)h * kHeadDim * kHeadDim, planes, threadIdx.x - 64, kThreads - 64);
+      split_transform(a, h, planes, threadIdx.x - 64, kThreads - 64);
       fence_proxy_async_smem();
     }
   }
@@ -377,8 +396,8 @@ bool input_map(CUtensorMap* m, const void* base, int hkv, int rows) {
 }  // namespace
 
 cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, const void* v_new, int n_new,
-                                      const int32_t* start_pos, const float* Tk, int32_t* status,
-                                      cudaStream_t stream) {
+                                      const int32_t* start_pos, const float* Tk, int tkind, int tblock,
+                                      int32_t* status, cudaStream_t stream) {
   TcArgs a{};
   a.num_kv_heads = c.num_kv_heads;
   a.total_rows = c.batch * n_new;
@@ -395,6 +414,8 @@ cudaError_t launch_quantize_append_tc(const wushkv_cache& c, const void* k_new, 
   a.ctas_per_head = cph;
   a.start_pos = start_pos;
   a.tk = Tk;
+  a.tkind = tkind;
+  a.tblock = tblock;
   a.k_codes = c.k_codes;
   a.v_codes = c.v_codes;
   a.k_meta = c.k_meta;

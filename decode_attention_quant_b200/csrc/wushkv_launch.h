@@ -19,6 +19,11 @@ cudaError_t launch_transform_query(const void* q, int q_dtype, int batch, int nu
                                    int num_kv_heads, const float* Tk_invT, float* q_out,
                                    cudaStream_t stream);
 
+// Query map by a structured transform's inverse-transpose (kind: wushkv_transform_kind).
+cudaError_t launch_transform_query_structured(const void* q, int q_dtype, int batch, int num_q_heads,
+                                              int num_kv_heads, int kind, int block, const float* data,
+                                              float* q_out, cudaStream_t stream);
+
 // Split count used when the caller passes num_splits = 0.
 int auto_num_splits(const wushkv_cache& c, int num_q_heads);
 size_t decode_workspace_bytes(const wushkv_cache& c, int num_q_heads, int num_splits);

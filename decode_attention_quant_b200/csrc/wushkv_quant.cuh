@@ -32,6 +32,33 @@ constexpr float kWidenDn = 0.999999046325683594f;  // 1 - 2^-20 (exact in fp32)
 constexpr float kWidenUp = 1.00000095367431641f;   // 1 + 2^-20 (exact in fp32)
 constexpr double kStepMargin = 1.0e-6;
 
+// Two fp32 values in one 64-bit register pair (element 0 in the low word) for the
+// sm_100a packed f32x2 arithmetic, which does two fp32 operations per instruction with
+// the same rounding as the scalar ones.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t x, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(x));
+}
+__device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fma2_rm(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t sub2_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 template <int BITS>
 __device__ __forceinline__ void put_code(uint32_t (&w)[4 * BITS], int i, uint32_t c) {
   const int o = BITS * i;
@@ -113,15 +140,33 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t
   constexpr int kHalf = 1 << (BITS - 1);
   constexpr int kMaxCode = (1 << BITS) - 1;
   const unsigned mask = __activemask();
+  // eight fp32 chains of 16 squares each (two per packed accumulator for bf16 rows, whose
+  // values are unpacked into fresh registers anyway)
   float s[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) s[k] = 0.f;
+  if constexpr (Loader::kBf16Exact) {
+    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll 1
-  for (int c = 0; c < kNumChunks; ++c) {
-    float v[kChunk];
-    ld(c, v);
+    for (int c = 0; c < kNumChunks; ++c) {
+      float v[kChunk];
+      ld(c, v);
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) s[i & 7] = fmaf(v[i], v[i], s[i & 7]);
+      for (int i = 0; i < kChunk / 2; ++i) {
+        const uint64_t p = pk2(v[2 * i], v[2 * i + 1]);
+        acc2[i & 3] = fma2_rn(p, p, acc2[i & 3]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) unpk2(acc2[k], s[2 * k], s[2 * k + 1]);
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < kNumChunks; ++c) {
+      float v[kChunk];
+      ld(c, v);
+#pragma unroll
+      for (int i = 0; i < kChunk; ++i) s[i & 7] = fmaf(v[i], v[i], s[i & 7]);
+    }
   }
   const double sum_fast = (((double)s[0] + (double)s[1]) + ((double)s[2] + (double)s[3])) +
                           (((double)s[4] + (double)s[5]) + ((double)s[6] + (double)s[7]));
@@ -147,7 +192,12 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t
   const float inv = (delta == 0.f || isinf(delta)) ? 0.f : __frcp_rn(delta);
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
+  // y = round-down(x * inv + 2^23 * 1.5 + 2^(b-1)) holds floor(x / Delta) + 2^(b-1) in its
+  // low mantissa bits; clamping y to [1.5 * 2^23, 1.5 * 2^23 + 2^b - 1] in fp32 leaves
+  // exactly the code there
   const float m = kMagic + (float)kHalf;
+  const float ylo = kMagic, yhi = kMagic + (float)kMaxCode;
+  const uint64_t m2 = pk2(m, m);
   if constexpr (Loader::kBf16Exact) {
 #pragma unroll 1
     for (int c = 0; c < kNumChunks; ++c) {
@@ -157,15 +207,19 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t
 #pragma unroll
       for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
-      for (int i = 0; i < kChunk; ++i) {
-        const float y = __fmaf_rd(v[i], v[i] < 0.f ? inv_dn : inv_up, m);
-        const int32_t code = min(max(f2i(y) - kMagicBits, 0), kMaxCode);
-        put_chunk_code<BITS>(wc, i, (uint32_t)code);
+      for (int i = 0; i < kChunk / 2; ++i) {
+        const uint64_t y2 = fma2_rm(pk2(v[2 * i], v[2 * i + 1]),
+                                    pk2(v[2 * i] < 0.f ? inv_dn : inv_up, v[2 * i + 1] < 0.f ? inv_dn : inv_up), m2);
+        float ya, yb;
+        unpk2(y2, ya, yb);
+        put_chunk_code<BITS>(wc, 2 * i, f2u(fminf(fmaxf(ya, ylo), yhi)) & (uint32_t)kMaxCode);
+        put_chunk_code<BITS>(wc, 2 * i + 1, f2u(fminf(fmaxf(yb, ylo), yhi)) & (uint32_t)kMaxCode);
       }
       store_chunk<BITS>(dst, c, wc);
     }
     return;
   }
+  const uint64_t dn2 = pk2(inv_dn, inv_dn), up2 = pk2(inv_up, inv_up);
   uint32_t mism = 0u;
 #pragma unroll 1
   for (int c = 0; c < kNumChunks; ++c) {
@@ -175,12 +229,16 @@ __device__ __forceinline__ void quest_quantize(Loader& ld, double alpha, uint8_t
 #pragma unroll
     for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
-      const float y1 = __fmaf_rd(v[i], inv_dn, m);
-      const float y2 = __fmaf_rd(v[i], inv_up, m);
-      mism |= f2u(y1) ^ f2u(y2);
-      const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-      put_chunk_code<BITS>(wc, i, (uint32_t)code);
+    for (int i = 0; i < kChunk / 2; ++i) {
+      const uint64_t p = pk2(v[2 * i], v[2 * i + 1]);
+      const uint64_t y1 = fma2_rm(p, dn2, m2);
+      const uint64_t y2 = fma2_rm(p, up2, m2);
+      const uint64_t dif = y1 ^ y2;
+      mism |= (uint32_t)dif | (uint32_t)(dif >> 32);
+      float ya, yb;
+      unpk2(y1, ya, yb);
+      put_chunk_code<BITS>(wc, 2 * i, f2u(fminf(fmaxf(ya, ylo), yhi)) & (uint32_t)kMaxCode);
+      put_chunk_code<BITS>(wc, 2 * i + 1, f2u(fminf(fmaxf(yb, ylo), yhi)) & (uint32_t)kMaxCode);
     }
     store_chunk<BITS>(dst, c, wc);
   }
@@ -218,6 +276,39 @@ __device__ __forceinline__ void select_update(float v, float (&lo)[KSEL], float 
   hi[0] = fmaxf(hi[0], v);
 }
 
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3f_q(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Three smallest (lo, ascending) and three largest (hi, descending) values so far, updated
+// with four more values at once: the four are sorted by a five-comparator network, then
+// each end is merged; the k-th smallest of two sorted lists A, B is the least over splits
+// i + j = k of max(A[i-1], B[j-1]) (and symmetrically for the largest).
+__device__ __forceinline__ void select_update4(float v0, float v1, float v2, float v3, float (&lo)[3],
+                                               float (&hi)[3]) {
+  float a = fminf(v0, v1), b = fmaxf(v0, v1), c = fminf(v2, v3), d = fmaxf(v2, v3);
+  const float s0 = fminf(a, c), t2 = fmaxf(a, c);
+  const float t1 = fminf(b, d), s3 = fmaxf(b, d);
+  const float s1 = fminf(t1, t2), s2 = fmaxf(t1, t2);     // s0 <= s1 <= s2 <= s3
+  const float n2 = fminf(min3f(lo[2], s2, fmaxf(lo[1], s0)), fmaxf(lo[0], s1));
+  const float n1 = min3f(lo[1], s1, fmaxf(lo[0], s0));
+  lo[0] = fminf(lo[0], s0);
+  lo[1] = n1;
+  lo[2] = n2;
+  const float m2 = fmaxf(max3f_q(hi[2], s1, fminf(hi[1], s3)), fminf(hi[0], s2));
+  const float m1 = max3f_q(hi[1], s2, fminf(hi[0], s3));
+  hi[0] = fmaxf(hi[0], s3);
+  hi[1] = m1;
+  hi[2] = m2;
+}
+
 template <int KSEL>
 __device__ __forceinline__ float pick(const float (&a)[KSEL], int idx) {
   float r = a[0];
@@ -237,18 +328,24 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
     lo_k[k] = __int_as_float(0x7f800000);
     hi_k[k] = __int_as_float(0xff800000);
   }
-  float fsum = 0.f;
+  static_assert(KSEL == 3, "the four-at-a-time selection keeps three values at each end");
+  uint64_t fsum2 = 0ull;                  // packed sum, only to detect NaN / Inf inputs
 #pragma unroll 1
   for (int c = 0; c < kNumChunks; ++c) {
     float v[kChunk];
     ld(c, v);
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
-      select_update<KSEL>(v[i], lo_k, hi_k);
-      fsum += v[i];
+    for (int i = 0; i < kChunk; i += 4) {
+      select_update4(v[i], v[i + 1], v[i + 2], v[i + 3], lo_k, hi_k);
+      fsum2 = fma2_rn(pk2(v[i], v[i + 1]), pk2(1.f, 1.f), fsum2);
+      fsum2 = fma2_rn(pk2(v[i + 2], v[i + 3]), pk2(1.f, 1.f), fsum2);
     }
   }
-  if (!isfinite(fsum)) flags |= WUSHKV_STATUS_NONFINITE;
+  {
+    float fa, fb;
+    unpk2(fsum2, fa, fb);
+    if (!isfinite(fa + fb)) flags |= WUSHKV_STATUS_NONFINITE;
+  }
   const float lo = pick<KSEL>(lo_k, rank_lo);
   const float hi = pick<KSEL>(hi_k, kHeadDim - 1 - rank_hi);
   const double scale_pre = ((double)hi - (double)lo) / (double)kMaxCode;
@@ -261,6 +358,10 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
   const float inv = (sc == 0.f || isinf(sc)) ? 0.f : __frcp_rn(sc);
   const float inv_dn = __fmul_rd(inv, kWidenDn);
   const float inv_up = __fmul_ru(inv, kWidenUp);
+  // y = rne((x - zero) * inv) + 1.5 * 2^23; clamped to [1.5 * 2^23, 1.5 * 2^23 + 2^b - 1]
+  // its low mantissa bits are the code
+  const uint64_t z2 = pk2(z, z), dn2 = pk2(inv_dn, inv_dn), up2 = pk2(inv_up, inv_up), m2 = pk2(kMagic, kMagic);
+  const float ylo = kMagic, yhi = kMagic + (float)kMaxCode;
   uint32_t mism = 0u;
 #pragma unroll 1
   for (int c = 0; c < kNumChunks; ++c) {
@@ -270,13 +371,16 @@ __device__ __forceinline__ void affine_quantize(Loader& ld, int rank_lo, int ran
 #pragma unroll
     for (int k = 0; k < BITS; ++k) wc[k] = 0u;
 #pragma unroll
-    for (int i = 0; i < kChunk; ++i) {
-      const float d = __fsub_rn(v[i], z);
-      const float y1 = __fmaf_rn(d, inv_dn, kMagic);
-      const float y2 = __fmaf_rn(d, inv_up, kMagic);
-      mism |= f2u(y1) ^ f2u(y2);
-      const int32_t code = min(max(f2i(y1) - kMagicBits, 0), kMaxCode);
-      put_chunk_code<BITS>(wc, i, (uint32_t)code);
+    for (int i = 0; i < kChunk / 2; ++i) {
+      const uint64_t d = sub2_rn(pk2(v[2 * i], v[2 * i + 1]), z2);
+      const uint64_t y1 = fma2_rn(d, dn2, m2);
+      const uint64_t y2 = fma2_rn(d, up2, m2);
+      const uint64_t dif = y1 ^ y2;
+      mism |= (uint32_t)dif | (uint32_t)(dif >> 32);
+      float ya, yb;
+      unpk2(y1, ya, yb);
+      put_chunk_code<BITS>(wc, 2 * i, f2u(fminf(fmaxf(ya, ylo), yhi)) & (uint32_t)kMaxCode);
+      put_chunk_code<BITS>(wc, 2 * i + 1, f2u(fminf(fmaxf(yb, ylo), yhi)) & (uint32_t)kMaxCode);
     }
     store_chunk<BITS>(dst, c, wc);
   }

@@ -178,16 +178,18 @@ typedef enum {
   WUSHKV_TRANSFORM_HADAMARD_DIAG = 3
 } wushkv_transform_kind;
 
-/* wushkv_quantize_append with a structured key transform: block-diagonal keys cost b
- * instead of 128 multiply-adds per channel, Hadamard-diagonal ones a scale and a
- * seven-stage butterfly.  kind is a wushkv_transform_kind; block is b for BLOCK_DIAG
- * (ignored otherwise); data is device fp32, 16-byte aligned, laid out as above.
- * DENSE takes every call wushkv_quantize_append takes.  The structured kinds are built
- * for decode-step appends (bf16, batch * n_new <= 64 token rows); other calls return
- * WUSHKV_ERR_UNSUPPORTED.  Results equal wushkv_quantize_append given the expanded
- * dense T_k up to the fp32 rounding of the transform; for BLOCK_DIAG they are
- * identical to the decode-step path given the expanded matrix.  Other arguments,
- * errors and status bits as wushkv_quantize_append. */
+/* wushkv_quantize_append with a structured key transform.  kind is a
+ * wushkv_transform_kind; block is b for BLOCK_DIAG (ignored otherwise); data is device
+ * fp32, 16-byte aligned, laid out as above.  DENSE takes every call
+ * wushkv_quantize_append takes.  The structured kinds take bf16 inputs: decode-step
+ * appends (batch * n_new <= 64 token rows) cost b instead of 128 multiply-adds per
+ * channel (block-diagonal) or a scale and a seven-stage butterfly (Hadamard-diagonal);
+ * larger appends expand the transform into the tensor-core kernel's exact bf16 parts
+ * of T_k and cost the same as a dense one.  fp32 inputs return WUSHKV_ERR_UNSUPPORTED.
+ * Results equal wushkv_quantize_append given the expanded dense T_k up to the fp32
+ * rounding of the transform; for BLOCK_DIAG they are identical to the dense path of the
+ * same size given the expanded matrix.  Other arguments, errors and status bits as
+ * wushkv_quantize_append. */
 WUSHKV_API int wushkv_quantize_append_structured(const wushkv_cache* cache, const void* k_new, const void* v_new,
                                       int32_t in_dtype, int32_t n_new, const int32_t* start_pos, int32_t kind,
                                       int32_t block, const float* data, int32_t* status, void* stream);
@@ -202,6 +204,21 @@ WUSHKV_API int wushkv_quantize_append_structured(const wushkv_cache* cache, cons
  *   q_out   : fp32 [batch][num_q_heads][128]; may not alias q. */
 WUSHKV_API int wushkv_transform_query(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
                            int32_t num_kv_heads, const float* Tk_invT, float* q_out, void* stream);
+
+/* wushkv_transform_query for the structured key transforms above: the query is mapped
+ * by T_k^{-T} of the head's KV head ([ai4s 6]: cheaper structured transforms), given as
+ *   DENSE         - data = T_k^{-T}, fp32 [Hkv][128][128] (exactly wushkv_transform_query);
+ *   BLOCK_DIAG    - data = the blocks of T_k^{-T}, fp32 [Hkv][128/b][b][b] (block j of T_k
+ *                   inverted and transposed, computed once per layer by the caller), b = block;
+ *   HADAMARD_DIAG - data = s, fp32 [Hkv][128], the same scales as the key transform
+ *                   (T_k^{-T} = H diag(1/s) / sqrt(128), since H / sqrt(128) is symmetric
+ *                   and orthogonal); every s must be nonzero.
+ * kind is a wushkv_transform_kind; block is 16, 32 or 64 for BLOCK_DIAG and ignored
+ * otherwise; data is device memory, 16-byte aligned.  Other arguments and errors as
+ * wushkv_transform_query. */
+WUSHKV_API int wushkv_transform_query_structured(const void* q, int32_t q_dtype, int32_t batch, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t kind, int32_t block, const float* data,
+                                      float* q_out, void* stream);
 
 /* Bytes of decode workspace needed for wushkv_decode_attention with the same
  * cache shape, num_q_heads and num_splits (0 = the automatic split count, else

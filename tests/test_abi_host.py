@@ -246,7 +246,32 @@ def test_append_structured_argument_checks():
     assert call(block=128) == _lib.ERR_UNSUPPORTED
     assert call(data=None) == _lib.ERR_INVALID
     assert call(data=0x80004) == _lib.ERR_MISALIGNED
-    assert call(n=33) == _lib.ERR_UNSUPPORTED            # not a decode-step append
+    assert call(n=0) == _lib.ERR_INVALID
     assert call(kind=3, dt=1) == _lib.ERR_UNSUPPORTED     # fp32 keys
     assert call(kind=1, data=None) == _lib.ERR_INVALID    # dense needs its matrix
     assert call(kind=1, dt=7) == _lib.ERR_UNSUPPORTED     # dense forwards to the plain append's checks
+
+
+def test_transform_query_structured_argument_checks():
+    lib = dq.library()
+    f = lib.wushkv_transform_query_structured
+    ok = (0x50000, 0, 2, 32, 8, 2, 32, 0x80000, 0x90000, None)
+
+    def call(**kw):
+        args = list(ok)
+        names = ["q", "dt", "b", "hq", "hkv", "kind", "block", "data", "out", "stream"]
+        for key, val in kw.items():
+            args[names.index(key)] = val
+        return f(*args)
+
+    assert call(kind=9) == _lib.ERR_UNSUPPORTED
+    assert call(block=8) == _lib.ERR_UNSUPPORTED
+    assert call(dt=5) == _lib.ERR_UNSUPPORTED
+    assert call(hq=20) == _lib.ERR_INVALID              # not a multiple of the KV heads
+    assert call(hq=24) == _lib.ERR_UNSUPPORTED          # group size 3
+    assert call(b=0) == _lib.ERR_INVALID
+    assert call(data=None) == _lib.ERR_INVALID
+    assert call(out=0x50000) == _lib.ERR_INVALID        # output may not alias q
+    assert call(data=0x80004) == _lib.ERR_MISALIGNED
+    assert call(kind=3, q=0x50008) == _lib.ERR_MISALIGNED
+    assert call(kind=1, data=None) == _lib.ERR_INVALID  # dense forwards to wushkv_transform_query
