@@ -47,6 +47,7 @@
 #include "tmap.h"
 #include "wushkv_common.cuh"
 #include "wushkv_launch.h"
+#include "wushkv_quant.cuh"
 
 namespace wushkv {
 namespace {
@@ -116,7 +117,6 @@ struct Misc {
   uint64_t full[4];           // stage filled (bulk copies)
   uint64_t kw;                // 4 token warps: key codes of the tile widened
   uint64_t pr;                // 4 token warps: probabilities written (value codes widened before)
-  uint64_t mx;                // 4 token warps: per-warp tile maxima published
   uint64_t kdone;             // score MMAs of the tile done
   uint64_t vdone;             // value MMAs of the tile done
   uint32_t tmem_base;
@@ -272,7 +272,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
     for (int s = 0; s < S; ++s) mbar_init(&ms->full[s], 1);
     mbar_init(&ms->kw, 4);
     mbar_init(&ms->pr, 4);
-    mbar_init(&ms->mx, 4);
     mbar_init(&ms->kdone, 1);
     mbar_init(&ms->vdone, 1);
     ms->abort = 0;
@@ -554,14 +553,30 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
             tmem_ld16(tmem + lanes + C::kColS + j * C::NK + c0, *reinterpret_cast<uint32_t(*)[16]>(d + c0));
           tmem_ld_wait();
         }
+        // |limb sum| <= 128 * 240 * 128, so two limbs combine exactly in int32; the fp32
+        // steps run on pairs of heads (packed f32x2 arithmetic, same rounding)
+        if constexpr (G % 2 == 0) {
+          const uint64_t ks2 = pk2(ks[j], ks[j]), kz2 = pk2(kz[j], kz[j]), big2 = pk2(65536.0f, 65536.0f);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          // |limb sum| <= 128 * 240 * 128, so two limbs combine exactly in int32
-          const int lo = (int)d[h] + (int)d[G + h] * 256;
-          const int hi = (int)d[2 * G + h] + (int)d[3 * G + h] * 256;
-          const float si = fmaf((float)hi, 65536.0f, (float)lo);
-          const float dot = fmaf(ks[j], si * c1[h], kz[j] * c2[h]);
-          s2[j][h] = valid[j] ? dot : -CUDART_INF_F;
+          for (int h = 0; h < G; h += 2) {
+            const int lo0 = (int)d[h] + (int)d[G + h] * 256, lo1 = (int)d[h + 1] + (int)d[G + h + 1] * 256;
+            const int hi0 = (int)d[2 * G + h] + (int)d[3 * G + h] * 256;
+            const int hi1 = (int)d[2 * G + h + 1] + (int)d[3 * G + h + 1] * 256;
+            const uint64_t si = fma2_rn(pk2((float)hi0, (float)hi1), big2, pk2((float)lo0, (float)lo1));
+            float a0, a1;
+            unpk2(fma2_rn(ks2, mul2_rn(si, pk2(c1[h], c1[h + 1])), mul2_rn(kz2, pk2(c2[h], c2[h + 1]))), a0, a1);
+            s2[j][h] = valid[j] ? a0 : -CUDART_INF_F;
+            s2[j][h + 1] = valid[j] ? a1 : -CUDART_INF_F;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const int lo = (int)d[h] + (int)d[G + h] * 256;
+            const int hi = (int)d[2 * G + h] + (int)d[3 * G + h] * 256;
+            const float si = fmaf((float)hi, 65536.0f, (float)lo);
+            const float dot = fmaf(ks[j], si * c1[h], kz[j] * c2[h]);
+            s2[j][h] = valid[j] ? dot : -CUDART_INF_F;
+          }
         }
       }
       // ---- tile maxima: per head the largest score; the largest value scale
@@ -574,9 +589,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
         const float vm = warp_max(fmaxf(vs[0], vs[1]));
         if (lane == 0) reinterpret_cast<float*>(&ms->red[u][32])[qd] = vm;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->mx);
-      ok = __all_sync(0xffffffffu, ok && mbar_wait(&ms->mx, u, abort));
+      named_barrier(kBarTok, 128);              // the four token warps' maxima are published
       const float4 v4 = ms->red[u][32];
       const float vmax = max3f(v4.x, v4.y, fmaxf(v4.z, v4.w));
       // limb scale: e * scale * vq <= 65520 (1 + 2^-21) < 65536 for e = 2^(s - mt) <= 1
@@ -601,13 +614,28 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
       for (int j = 0; j < 2; ++j) {
         const float vsq = vs[j] * vq;
         uint32_t pb[G];
+        // round e * scale * vq to an integer <= 65535 held in the low 16 bits of the float's
+        // pattern; pairs of heads share the packed f32x2 steps
+        if constexpr (G % 2 == 0) {
+          const uint64_t vz2 = pk2(vz[j], vz[j]), vsq2 = pk2(vsq, vsq), mg2 = pk2(12582912.0f, 12582912.0f);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float e = ex2_approx(s2[j][h] - mt[h]);
-          lt[h] += e;
-          zt[h] = fmaf(e, vz[j], zt[h]);
-          // round to an integer <= 65535 held in the low 16 bits of the float's pattern
-          pb[h] = __float_as_uint(fmaf(e, vsq, 12582912.0f));
+          for (int h = 0; h < G; h += 2) {
+            const uint64_t e2 = pk2(ex2_approx(s2[j][h] - mt[h]), ex2_approx(s2[j][h + 1] - mt[h + 1]));
+            unpk2(add2_rn(pk2(lt[h], lt[h + 1]), e2), lt[h], lt[h + 1]);
+            unpk2(fma2_rn(e2, vz2, pk2(zt[h], zt[h + 1])), zt[h], zt[h + 1]);
+            float p0, p1;
+            unpk2(fma2_rn(e2, vsq2, mg2), p0, p1);
+            pb[h] = __float_as_uint(p0);
+            pb[h + 1] = __float_as_uint(p1);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float e = ex2_approx(s2[j][h] - mt[h]);
+            lt[h] += e;
+            zt[h] = fmaf(e, vz[j], zt[h]);
+            pb[h] = __float_as_uint(fmaf(e, vsq, 12582912.0f));
+          }
         }
         uint8_t* bcol = bv + j * C::NV * 128 + r * 16;
 #pragma unroll
@@ -822,6 +850,12 @@ int auto_num_splits(const wushkv_cache& c, int num_q_heads) {
     if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
   }
   return best;
+}
+
+// Combine of log2-domain split partials ([rows][splits][132]) into out [rows][128].
+cudaError_t launch_combine_partials(const float* ws, int rows, int num_splits, float* out, cudaStream_t stream) {
+  combine_log2_kernel<<<rows, kHeadDim, 0, stream>>>(ws, num_splits, out);
+  return cudaGetLastError();
 }
 
 size_t decode_workspace_bytes(const wushkv_cache& c, int num_q_heads, int num_splits) {

@@ -160,24 +160,11 @@ def test_paged_layout_accepted():
 def test_chunk_workspace_and_argument_checks():
     lib = dq.library()
     d = _desc()
-    # layout: prefix lengths, the decode pass's own output, folded queries and split partials
-    # of each pass (16 rows per KV head per pass), each rounded up to 64 floats
+    # layout: one partial (m, l, pad, pad, o[128]) per (sequence, chunk query, query head, split)
     def floats(hq, n_q, splits):
-        r64 = lambda n: -(-n // 64) * 64
-        rows = n_q * (hq // 2)
-        total = r64(2) + r64(2 * 2 * 16 * 128)
-        passes = []
-        while rows > 0:
-            gf = 1
-            while gf < min(rows, 16):
-                gf *= 2
-            passes.append(gf)
-            rows -= 16
-        total += sum(r64(2 * 2 * gf * 128) for gf in passes)
-        total += sum(r64(2 * 2 * gf * splits * 132) for gf in passes)
-        return total
-    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 16, 3) == 4 * floats(4, 16, 3) == 301312
-    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 3, 3) == 4 * floats(4, 3, 3) == 100096
+        return 2 * n_q * hq * splits * 132
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 16, 3) == 4 * floats(4, 16, 3) == 202752
+    assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 3, 3) == 4 * floats(4, 3, 3) == 38016
     assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 0, 0) == 0
     assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 4, 17, 0) == 0
     assert lib.wushkv_chunk_workspace_bytes(ctypes.byref(d), 6, 4, 0) == 0

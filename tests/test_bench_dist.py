@@ -47,10 +47,10 @@ def test_two_gloo_ranks_agree_on_max_and_reference_runs_on_rank0_only():
 
 
 def test_chunk_roofline_helpers():
-    """FLOP count of the chunk-attention sub-benchmark and the int8 tensor peak it is
+    """FLOP count of the chunk-attention sub-benchmark and the fp16 tensor peak it is
     compared with (host logic only)."""
     import bench
     # Qwen3-32B-shaped layer: 32 sequences x 16 queries x 64 heads x 8192 positions, 512 FLOPs each
     assert bench.chunk_flops(32, 16, 64, 8192) == 512 * 32 * 16 * 64 * 8192 == 137438953472
-    peak, kind = bench._int8_tensor_peak()
-    assert peak > 1000.0 and "x 2" in kind
+    peak, kind = bench._f16_tensor_peak()
+    assert peak > 1000.0 and "fp16" in kind

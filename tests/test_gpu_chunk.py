@@ -67,10 +67,35 @@ def test_chunk_matches_oracle(kind, bits, hq, hkv, n_q, ctx):
                 assert np.all(got[b, i] == 0), (b, i)
 
 
+@pytest.mark.parametrize("kind,bits,hq,hkv", [(0, 2, 8, 2), (1, 4, 16, 2), (0, 3, 4, 1)])
+def test_chunk_multi_tile_ctas(kind, bits, hq, hkv):
+    """One CTA walks many 128-position tiles (num_splits 1 and 2): double-buffered
+    operands, O accumulated across tiles, and the running reference moving for some rows
+    of a warp but not for others (queries scaled up so that tile maxima spread by more
+    than 2^8)."""
+    n_q, bsz, cap = 16, 2, 1000
+    c = gen.random_cache(bsz, hkv, cap, kind, bits, seed=31 + bits, device="cpu")
+    cache = dq.PackedCache(bsz, hkv, cap, kind, bits, tensors={k: v.cuda() for k, v in c.items()})
+    q = (_chunk_queries(bsz, n_q, hq, seed=40 + hq) * 4.0).contiguous()
+    ctx = [1000, 611]
+    cn = {name: t.numpy() for name, t in c.items()}
+    cn["k_meta"] = cn["k_meta"].view(np.uint16)
+    cn["v_meta"] = cn["v_meta"].view(np.uint16)
+    ref = orc.chunk_attention(cn, q.numpy().astype(np.float64), ctx, TAU, kind, bits, hkv)
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    for s in (1, 2):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        got = dq.chunk_attention(cache, q.cuda(), ctx_t, TAU, num_splits=s, status=st).cpu().numpy()
+        assert st.item() == 0
+        ma, rl = gu.attention_errors(got, ref)
+        print(f"kind={kind} bits={bits} g={hq // hkv} splits={s}: max-abs {ma:.3e} rel-L2 {rl:.3e}")
+        assert ma <= MAX_ABS and rl <= REL_L2
+
+
 def test_chunk_last_query_and_splits():
-    """The chunk's last query is the decode query at the same context; the prefix split
-    count changes results only at the decode kernel's rounding level; contexts above
-    the capacity are clamped with the overflow bit."""
+    """The chunk's last query is the decode query at the same context; the split count
+    changes results only at fp32 rounding level; contexts above the capacity are
+    clamped with the overflow bit."""
     kind, bits, hq, hkv, n_q = 1, 2, 8, 2, 16
     bsz, cap = 3, 1100
     c = gen.random_cache(bsz, hkv, cap, kind, bits, seed=15, device="cpu")
@@ -80,12 +105,10 @@ def test_chunk_last_query_and_splits():
     outs = [dq.chunk_attention(cache, q, ctx, TAU, num_splits=s) for s in (0, 1, 3, 7)]
     for o in outs[1:]:
         assert torch.allclose(o, outs[0], rtol=0, atol=5e-5), (o - outs[0]).abs().max()
-    # The last query through the decode call: both match the oracle at the bar, and they
-    # differ from each other only by the decode kernel's 16-bit probability limbs
-    # (rounding <= 2^-17 of the tile maximum per term; over a 256-token tile with random
-    # signs about 16 * 2^-17 * max|v_hat|, max|v_hat| < 4 here: 2^-11).
+    # The last query through the decode call: the two kernels share no arithmetic (the
+    # decode kernel rounds probabilities to 16-bit limbs, the chunk kernel carries them
+    # as fp16 hi + lo), so each is held to the oracle at the bar.
     dec = dq.decode_attention(cache, q[:, n_q - 1].contiguous(), ctx, TAU)
-    assert torch.allclose(outs[0][:, n_q - 1], dec, rtol=0, atol=2.0 ** -11), (outs[0][:, n_q - 1] - dec).abs().max()
     cn = {name: t.numpy() for name, t in c.items()}
     cn["k_meta"] = cn["k_meta"].view(np.uint16)
     cn["v_meta"] = cn["v_meta"].view(np.uint16)
