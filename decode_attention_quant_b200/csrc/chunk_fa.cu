@@ -7,21 +7,30 @@
 // p_i = ctx - n_q + i (ctx = min(ctx_len[b], capacity)) and attends positions 0 .. p_i.
 //
 // One CTA = (split of the positions, KV head, block of 128 folded rows, sequence); row
-// f = i * g + h is query i of head h.  Per 128-position tile:
-//   converters (warps 0-3, thread = position): packed K and V codes -> exact fp16 codes in
-//     the 128-byte-swizzled layout both MMAs read, plus the tile's fp16 meta as fp32;
-//   MMA issuer (warp 12): S = Q' K^T as two fp16 MMAs (q' split into fp16 hi + lo, so the
-//     products carry 22 bits of q'; codes are exact), fp32 accumulation in tensor memory;
-//     then O += P V with P' = p * scale split the same way (P in tensor memory);
+// f = i * g + h is query i of head h.  512 threads; per 128-position tile:
+//   converters (warps 0-3): load the tile's packed K and V codes and meta one tile ahead
+//     (lane 4i + k takes quarter k of the packed rows of positions i, 8 + i, ...; thread
+//     t the meta of position t), turn the codes into exact fp16 (the code ORed into the
+//     mantissa of 1024, minus 1024; fp16 subnormals would save the subtraction, but the
+//     MMAs lose precision on subnormal operands) and store them with stmatrix into a
+//     three-stage ring of 128-byte-swizzled K-major operands: keys as [position][slot],
+//     values transposed as [slot][position] (a K-major B runs the value MMAs about 1.7x
+//     faster than an MN-major one); the meta as fp32;
+//   issuer (warp 12, one thread): S = Q' K^T as two fp16 MMAs with q' in tensor memory
+//     (split into fp16 hi + lo, so the products carry 22 bits of q'), fp32 accumulation;
+//     then O += P' V as two fp16 MMAs with P' in tensor memory;
 //   softmax (warps 4-11, thread = row and half of the tile's positions): scores
 //     s = tau log2e (scale_t q'.c + zero_t sum q') in the log2 domain, causal mask, the
 //     tile maximum, e = 2^(s - m) against a running reference m that moves only when the
-//     maximum passes it by 8 (then O, l and z are rescaled), sums l = sum e and
-//     z = sum e * zero, and P' = e * scale in fp16 hi + lo.
-// The split partial (m, l, o + z) goes to the workspace; a combine pass merges splits.
-// 2- and 4-bit codes are converted in pairs straight from their packed words, which
-// orders the channels of each 16 (8) channel group as (k, k + 8) ((k, k + 4)) pairs; the
-// query and the output use the same order.
+//     maximum passes it by 2^8 (then O, l and z are rescaled), l = sum e, z = sum e * zero,
+//     and P' = e * scale * 2^-E in fp16 hi + lo.
+// The softmax warpgroups take most of the register file (setmaxnreg); warps 13-15 only
+// give theirs up.  E is the running maximum exponent of the value scales seen so far
+// (from the converters), which keeps P' <= 2^8 inside fp16 for any scale; O is rescaled
+// by an exact power of two when it grows.  The split partial (m, l, O 2^E + z) goes to
+// the workspace; a combine pass merges splits.  Codes are converted in pairs straight
+// from the lane's quarter of the packed row, which permutes the channels (slot_channel);
+// the query and the output use the same order.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -29,6 +38,7 @@
 #include "tmap.h"
 #include "wushkv_common.cuh"
 #include "wushkv_launch.h"
+#include "wushkv_quant.cuh"
 
 namespace wushkv {
 namespace {
@@ -37,48 +47,50 @@ using namespace sm100;
 
 constexpr int kN = 128;                         // cached positions per tile
 constexpr int kRows = 128;                      // folded rows per CTA = TMEM lanes
+constexpr int kStages = 3;                      // K/V operand ring
 constexpr int kConvWarps = 4;
 constexpr int kSoftWarps = 8;
 constexpr int kMmaWarp = kConvWarps + kSoftWarps;
-constexpr int kThreads = 32 * (kMmaWarp + 1);   // 416
+constexpr int kThreads = 512;                   // four warpgroups
+constexpr int kRegsConv = 104, kRegsSoft = 184, kRegsMma = 40;
+static_assert(128 * kRegsConv + 256 * kRegsSoft + 128 * kRegsMma <= 65536, "register split over the launch's");
 constexpr int kPartialStride = 132;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;                   // log2 headroom of the running reference
 constexpr int kHalfBytes = 16384;               // [128 rows][64 x 16-bit], 128-byte swizzled
+constexpr int kNoScale = -126;                  // value-scale exponent before any valid position
 
-constexpr int kColS = 0;                        // 2 x 128 columns: double-buffered scores
+constexpr int kColS = 0;                        // 128 columns: scores
+constexpr int kColQ = 128;                      // q' hi (64 columns) then q' lo (64)
 constexpr int kColP = 256;                      // P' hi (64 columns) then P' lo (64)
 constexpr int kColO = 384;                      // 128 columns
 constexpr int kCols = 512;
 
 struct FaBars {
-  uint64_t full, cfree;            // code stage: filled by TMA / read by the converters
-  uint64_t conv[2], kvfree[2];     // operand buffers: written / released by their MMAs
-  uint64_t sfull[2], sfree[2];     // score buffers: computed / read by the softmax warps
-  uint64_t pfull, pvdone;          // P' written (and O rescaled) / PV MMA done
+  uint64_t conv[kStages], kvfree[kStages];   // operand stages: written / released by the PV MMAs
+  uint64_t sfull, sfree;                      // scores: computed / read by the softmax warps
+  uint64_t pfull, pvdone;                     // P' written (and O rescaled) / PV MMAs done
+  uint64_t drain;                             // MMAs in flight at a timeout
   uint32_t tmem_base;
   int abort;
 };
 
-template <int BITS>
-struct FaCfg {
-  static constexpr int kCode = 16 * BITS;
-  static constexpr int kStage = 2 * kN * kCode;              // K then V codes of one tile
-  static constexpr int kOffQh = 0;                            // A of S: q' hi [2 halves][128 rows][128 B]
-  static constexpr int kOffQl = kOffQh + 2 * kHalfBytes;      // q' lo
-  static constexpr int kOffKb = kOffQl + 2 * kHalfBytes;      // B of S: 2 buffers [2 halves][128 pos][128 B]
-  static constexpr int kOffVb = kOffKb + 4 * kHalfBytes;      // B of PV: 2 buffers, same layout (MN-major)
-  static constexpr int kOffStage = kOffVb + 4 * kHalfBytes;
-  static constexpr int kOffMeta = kOffStage + kStage;         // 2 buffers of {ks, kz, vs, vz}[128] + 4 mask words
-  static constexpr int kMetaBytes = 4 * kN * 4 + 16;
-  static constexpr int kOffRow = kOffMeta + 2 * kMetaBytes;   // row exchange [2][2][128] + [2][128] x 2
-  static constexpr int kOffBar = kOffRow + 8 * kRows * 4;
-  static constexpr int kSmem = kOffBar + (int)sizeof(FaBars) + 1024;
-  static_assert(kOffStage % 1024 == 0, "TMA boxes need 1 KB alignment");
-  static_assert(kSmem <= 227 * 1024, "one CTA per SM");
-};
+// Shared memory (operand stages 1 KB aligned for the 128-byte swizzle).
+constexpr int kOffKb = 0;                                  // B of S: [stage][2 halves][128 pos][128 B]
+constexpr int kOffVb = kOffKb + kStages * 2 * kHalfBytes;  // B of PV: [stage][2 halves][128 slots][128 B]
+constexpr int kOffMeta = kOffVb + kStages * 2 * kHalfBytes;
+// per stage: ks, kz, vs * 2^-E, vz [128] fp32; 4 validity words; E; padding
+constexpr int kMetaWords = 4 * kN + 8;
+constexpr int kMetaBytes = 4 * kMetaWords;
+constexpr int kOffRow = kOffMeta + kStages * kMetaBytes;   // row exchange [8][128] fp32
+constexpr int kOffScl = kOffRow + 8 * kRows * 4;           // converter warps' scale maxima [stage][4]
+constexpr int kOffBar = kOffScl + 64;
+constexpr int kSmem = kOffBar + (int)sizeof(FaBars) + 1024;
+static_assert(kSmem <= 227 * 1024, "one CTA per SM");
 
 struct FaArgs {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
   const uint16_t* k_meta;
   const uint16_t* v_meta;
   CacheRows rows;
@@ -86,32 +98,43 @@ struct FaArgs {
   const int32_t* ctx_len;
   float* ws;                   // partials [(b, i, h)][splits][132]
   int32_t* status;
-  int n_q, hq, hkv, capacity, num_splits, row_blocks, box_rows;
+  int n_q, hq, hkv, capacity, num_splits, row_blocks;
   float scale_log2;            // softmax scale * log2 e
 };
 
-// Channel held by slot s of a converted 128-value row (see the header).
+// Channel held by slot s (of 128) of a converted row.  Slot pair (8c + 2k, 8c + 2k + 1)
+// is pair c of quarter k of the packed row: 2-bit words 2k, 2k + 1 hold channels
+// 32k .. 32k + 31, pair c = word 2k + c / 8 shifted by 2 (c mod 8), so channels
+// (16 (2k + c / 8) + c mod 8, + 8); 4-bit words 4k .. 4k + 3, pair c = word 4k + c / 4
+// shifted by 4 (c mod 4): channels (8 (4k + c / 4) + c mod 4, + 4); 3-bit bits 96k ..
+// 96k + 95 hold channels 32k .. 32k + 31 in order.
 template <int BITS>
 __host__ __device__ __forceinline__ int slot_channel(int s) {
-  if (BITS == 2) return (s & ~15) | ((s >> 1) & 7) | ((s & 1) << 3);
-  if (BITS == 4) return (s & ~7) | ((s >> 1) & 3) | ((s & 1) << 2);
-  return s;
+  const int k = (s >> 1) & 3, c = s >> 3, e = s & 1;
+  if (BITS == 2) return 32 * k + 16 * (c >> 3) + (c & 7) + 8 * e;
+  if (BITS == 4) return 32 * k + 8 * (c >> 2) + (c & 3) + 4 * e;
+  return 32 * k + 2 * c + e;
 }
 
-// TMA swizzle of a stage's code rows (as the decode kernel's tensor maps lay them out).
+// Words of quarter k of a packed row: 2-bit 2, 3-bit 3, 4-bit 4.
 template <int BITS>
-__device__ __forceinline__ int stage_swizzle(int row) {
-  return BITS == 2 ? ((row >> 2) & 1) : BITS == 4 ? ((row >> 1) & 3) : 0;
-}
+struct Quarter {
+  static constexpr int W = BITS;
+  uint32_t k[W], v[W];
+};
 
 template <int BITS>
-__device__ __forceinline__ void load_code_row(const uint8_t* tile, int row, uint32_t (&w)[4 * BITS]) {
-  const uint8_t* p = tile + row * (16 * BITS);
-  const int sw = stage_swizzle<BITS>(row);
+__device__ __forceinline__ void load_quarter(const uint8_t* codes, long long row, int kq, uint32_t (&w)[BITS]) {
+  const uint8_t* p = codes + row * (16 * BITS) + 4 * BITS * kq;
+  if (BITS == 2) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    w[0] = v.x; w[1] = v.y;
+  } else if (BITS == 4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else {
 #pragma unroll
-  for (int q = 0; q < BITS; ++q) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p + 16 * (q ^ sw));
-    w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    for (int q = 0; q < BITS; ++q) w[q] = __ldg(reinterpret_cast<const uint32_t*>(p) + q);
   }
 }
 
@@ -122,28 +145,15 @@ __device__ __forceinline__ uint32_t unbias2(uint32_t x) {
   return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// Word j (slots 2j, 2j + 1) of a packed row's 128 codes as an fp16 pair, slot order.
+// Pair c of a quarter as an exact fp16 pair (slot order, see slot_channel).
 template <int BITS>
-__device__ __forceinline__ uint32_t code_pair_f16(const uint32_t (&w)[4 * BITS], int j) {
-  if (BITS == 2) return unbias2(((w[j >> 3] >> (2 * (j & 7))) & 0x00030003u) | 0x64006400u);
-  if (BITS == 4) return unbias2(((w[j >> 2] >> (4 * (j & 3))) & 0x000F000Fu) | 0x64006400u);
-  const int bit = 6 * j, wi = bit >> 5, sh = bit & 31;   // channels 2j, 2j + 1 at bits 6j .. 6j + 5
-  const uint32_t hi = (wi + 1 < 4 * BITS) ? w[wi + 1] : 0u;
+__device__ __forceinline__ uint32_t code_pair_f16(const uint32_t (&w)[BITS], int c) {
+  if (BITS == 2) return unbias2(((w[c >> 3] >> (2 * (c & 7))) & 0x00030003u) | 0x64006400u);
+  if (BITS == 4) return unbias2(((w[c >> 2] >> (4 * (c & 3))) & 0x000F000Fu) | 0x64006400u);
+  const int bit = 6 * c, wi = bit >> 5, sh = bit & 31;   // channels 2c, 2c + 1 of the quarter
+  const uint32_t hi = (wi + 1 < BITS) ? w[wi + 1] : 0u;
   const uint32_t f = __funnelshift_r(w[wi], hi, sh);
   return unbias2(((f & 7u) | ((f & 0x38u) << 13)) | 0x64006400u);
-}
-
-// A packed row's codes as exact fp16 in slot order, stored as row r of a [2 halves][128
-// rows][128 B] 128-byte-swizzled operand, one 16-byte chunk at a time.
-template <int BITS>
-__device__ __forceinline__ void store_code_row(uint8_t* base, int r, const uint32_t (&w)[4 * BITS]) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const uint32_t x0 = code_pair_f16<BITS>(w, 4 * c), x1 = code_pair_f16<BITS>(w, 4 * c + 1);
-    const uint32_t x2 = code_pair_f16<BITS>(w, 4 * c + 2), x3 = code_pair_f16<BITS>(w, 4 * c + 3);
-    *reinterpret_cast<uint4*>(base + (c >> 3) * kHalfBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)) =
-        make_uint4(x0, x1, x2, x3);
-  }
 }
 
 template <int KIND>
@@ -157,23 +167,70 @@ __device__ __forceinline__ void meta_of(uint32_t raw, int bits, float& scale, fl
   }
 }
 
+// fp32 2^e for e in [-126, 127] (exact)
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
+// The raw meta of one position (zero where the position is not valid).
+template <int KIND>
+struct PosMeta {
+  uint32_t km, vm;
+  bool valid;
+
+  __device__ __forceinline__ void load(const FaArgs& a, int b, int kv, int pos, int ctx) {
+    valid = false;
+    km = 0u;
+    vm = 0u;
+    if (pos < ctx) {
+      const long long row = a.rows.row(b, kv, pos);
+      if (row >= 0) {
+        valid = true;
+        if (KIND == WUSHKV_QUEST_INT) {
+          km = __ldg(a.k_meta + row);
+          vm = __ldg(a.v_meta + row);
+        } else {
+          km = __ldg(reinterpret_cast<const uint32_t*>(a.k_meta) + row);
+          vm = __ldg(reinterpret_cast<const uint32_t*>(a.v_meta) + row);
+        }
+      } else {
+        report(a.status, WUSHKV_STATUS_BAD_PAGE);
+      }
+    }
+  }
+};
+
+// Quarter kq of the K and V rows of positions base + 8m (m = 0..3), zero where not valid.
+template <int BITS>
+__device__ __forceinline__ void load_quarters(const FaArgs& a, int b, int kv, int base, int ctx, int kq,
+                                              Quarter<BITS> (&f)[4]) {
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int pos = base + 8 * m;
+    long long row = -1;
+    if (pos < ctx) row = a.rows.row(b, kv, pos);
+    if (row >= 0) {
+      load_quarter<BITS>(a.k_codes, row, kq, f[m].k);
+      load_quarter<BITS>(a.v_codes, row, kq, f[m].v);
+    } else {
+#pragma unroll
+      for (int q = 0; q < BITS; ++q) { f[m].k[q] = 0u; f[m].v[q] = 0u; }
+    }
+  }
+}
+
 template <int BITS, int KIND>
-__global__ void __launch_bounds__(kThreads, 1)
-    chunk_fa_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, FaArgs a) {
-  using C = FaCfg<BITS>;
+__global__ void __launch_bounds__(kThreads, 1) chunk_fa_kernel(const FaArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qh = smem + C::kOffQh;
-  uint8_t* ql = smem + C::kOffQl;
-  uint8_t* kb = smem + C::kOffKb;
-  uint8_t* vb = smem + C::kOffVb;
-  uint8_t* stage = smem + C::kOffStage;
-  uint8_t* meta = smem + C::kOffMeta;
-  float* rowx = reinterpret_cast<float*>(smem + C::kOffRow);
-  FaBars* bars = reinterpret_cast<FaBars*>(smem + C::kOffBar);
+  uint8_t* kb = smem + kOffKb;
+  uint8_t* vb = smem + kOffVb;
+  float* meta = reinterpret_cast<float*>(smem + kOffMeta);
+  float* rowx = reinterpret_cast<float*>(smem + kOffRow);
+  uint32_t* sclx = reinterpret_cast<uint32_t*>(smem + kOffScl);
+  FaBars* bars = reinterpret_cast<FaBars*>(smem + kOffBar);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
   const int split = blockIdx.x, kv = blockIdx.y / a.row_blocks, rb = blockIdx.y % a.row_blocks, b = blockIdx.z;
   const int g = a.hq / a.hkv, R = a.n_q * g;
   int ctx = __ldg(a.ctx_len + b);
@@ -186,20 +243,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int per = (tiles_all + a.num_splits - 1) / a.num_splits;
   const int tile0 = split * per;
   const int n = max(0, min(per, tiles_all - tile0));
-  const int pair = b * a.hkv + kv;
-  const bool paged = a.rows.block_table != nullptr;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->full, 1);
-    mbar_init(&bars->cfree, kConvWarps);
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < kStages; ++j) {
       mbar_init(&bars->conv[j], kConvWarps);
       mbar_init(&bars->kvfree[j], 1);
-      mbar_init(&bars->sfull[j], 1);
-      mbar_init(&bars->sfree[j], kSoftWarps);
     }
+    mbar_init(&bars->sfull, 1);
+    mbar_init(&bars->sfree, kSoftWarps);
     mbar_init(&bars->pfull, kSoftWarps);
     mbar_init(&bars->pvdone, 1);
+    mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -207,64 +261,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&bars->tmem_base, kCols);
     tmem_relinquish();
   }
-
-  // Warp 12: the copies of tile i's K and V code rows into the stage (one 3-D box per
-  // side, or one per page the tile touches; rows past the capacity arrive as zeros).
-  int issued = 0;
-  auto issue_load = [&](int i) {
-    ++issued;
-    const int t0 = (tile0 + i) * kN;
-    uint8_t* kdst = stage;
-    uint8_t* vdst = stage + kN * C::kCode;
-    if (lane == 0) mbar_arrive_expect_tx(&bars->full, C::kStage);
-    __syncwarp();
-    if (!paged) {
-      if (lane == 0) {
-        tma_load_3d(kdst, &kmap, &bars->full, 0, t0, pair);
-        tma_load_3d(vdst, &vmap, &bars->full, 0, t0, pair);
-      }
-    } else if (lane < kN / a.box_rows) {
-      const int t = t0 + lane * a.box_rows;
-      const int page = t < a.capacity
-                           ? __ldg(a.rows.block_table + (size_t)b * a.rows.pages_per_seq + (t >> a.rows.page_shift))
-                           : -1;
-      const bool in = page >= 0 && page < a.rows.num_pages;
-      const int c1 = in ? (t & ((1 << a.rows.page_shift) - 1)) : 0;
-      const int c2 = in ? page * a.hkv + kv : a.rows.num_pages * a.hkv;
-      const int off = lane * a.box_rows * C::kCode;
-      tma_load_3d(kdst + off, &kmap, &bars->full, 0, c1, c2);
-      tma_load_3d(vdst + off, &vmap, &bars->full, 0, c1, c2);
-    }
-  };
-  if (warp == kMmaWarp) {
-    __syncwarp();
-    tma_prefetch(&kmap);
-    tma_prefetch(&vmap);
-    if (n > 0) issue_load(0);
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
 
   // Softmax warps: row r of this block, half hf of each tile's positions (and of the
   // query's slots while preparing the query operand).
-  const int sw = warp - kConvWarps;
   const int r = 32 * (warp & 3) + lane;
-  const int hf = sw >> 2;
+  const int hf = (warp - kConvWarps) >> 2;
   const int f = rb * kRows + r;
   const bool row_ok = f < R;
   const int qi = row_ok ? f / g : 0;
   const int qh_idx = row_ok ? kv * g + f % g : 0;
   const int p_last = ctx - a.n_q + qi;                 // last visible position of this row
-  float rowc = 0.f, qs = 0.f;                            // per row: tau log2e / sigma, tau log2e sum q'
+  const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
   const uint32_t bar_pair = 2 + (warp & 3);              // the two softmax warps of a lane quarter
+  float rowc = 0.f, qs = 0.f;                            // per row: tau log2e / sigma, tau log2e sum q'
   if (warp >= kConvWarps && warp < kMmaWarp) {
-    // q' row (fp32) -> sigma q' in fp16 hi + lo, slots 64 hf .. 64 hf + 63
-    const float* qrow = a.q + (((size_t)b * a.n_q + qi) * a.hq + qh_idx) * kHeadDim;
-    float v[64];
+    // q' row: slots 64 hf .. 64 hf + 63 hold channels 32k + 16 hf .. 32k + 16 hf + 15
+    // (k = 0..3), loaded as 16 float4 -> sigma q' in fp16 hi + lo, slot order, into
+    // tensor memory as the A operand of the score MMAs
+    const float4* qrow = reinterpret_cast<const float4*>(a.q + (((size_t)b * a.n_q + qi) * a.hq + qh_idx) * kHeadDim);
+    float ch[64];                                        // ch[16k + j] = channel 32k + 16 hf + j
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float4 v4 = row_ok ? __ldg(qrow + 8 * (m >> 2) + 4 * hf + (m & 3)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ch[4 * m] = v4.x; ch[4 * m + 1] = v4.y; ch[4 * m + 2] = v4.z; ch[4 * m + 3] = v4.w;
+    }
     float mx = 0.f, sm = 0.f;
 #pragma unroll
     for (int s = 0; s < 64; ++s) {
-      v[s] = row_ok ? __ldg(qrow + slot_channel<BITS>(64 * hf + s)) : 0.f;
-      mx = fmaxf(mx, fabsf(v[s]));
-      sm += v[s];
+      mx = fmaxf(mx, fabsf(ch[s]));
+      sm += ch[s];
     }
     rowx[hf * kRows + r] = mx;
     rowx[2 * kRows + hf * kRows + r] = sm;
@@ -277,90 +306,113 @@ __global__ void __launch_bounds__(kThreads, 1)
     rowc = a.scale_log2 / sigma;
     qs = sm * a.scale_log2;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {                        // 16-byte chunk c: slots 8c .. 8c + 7
-      uint32_t x[4], y[4];
+    for (int c = 0; c < 2; ++c) {                        // slots 32c .. 32c + 31 -> 16 columns
+      uint32_t x[16], y[16];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float x0 = v[8 * c + 2 * k] * sigma, x1 = v[8 * c + 2 * k + 1] * sigma;
+      for (int k = 0; k < 16; ++k) {
+        // slot 64 hf + s0 holds channel slot_channel(s0) + 16 hf
+        const int s0 = 32 * c + 2 * k;
+        const int c0 = slot_channel<BITS>(s0), c1 = slot_channel<BITS>(s0 + 1);
+        const float x0 = ch[16 * (c0 >> 5) + (c0 & 15)] * sigma, x1 = ch[16 * (c1 >> 5) + (c1 & 15)] * sigma;
         const __half2 h2 = __floats2half2_rn(x0, x1);
         const float2 hb = __half22float2(h2);
         const __half2 l2 = __floats2half2_rn(x0 - hb.x, x1 - hb.y);
         x[k] = *reinterpret_cast<const uint32_t*>(&h2);
         y[k] = *reinterpret_cast<const uint32_t*>(&l2);
       }
-      const int off = hf * kHalfBytes + r * 128 + ((c ^ (r & 7)) << 4);
-      *reinterpret_cast<uint4*>(qh + off) = make_uint4(x[0], x[1], x[2], x[3]);
-      *reinterpret_cast<uint4*>(ql + off) = make_uint4(y[0], y[1], y[2], y[3]);
+      tmem_st16(tmem + lanes + kColQ + 32 * hf + 16 * c, x);
+      tmem_st16(tmem + lanes + kColQ + 64 + 32 * hf + 16 * c, y);
     }
-    fence_proxy_async_smem();
+    tmem_st_wait();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
 
+  // Each role runs entirely inside its branch, which starts by resizing its registers.
   if (warp < kConvWarps) {
     // ------------------------------------------------------------- converters
-    const int t = threadIdx.x;                           // position t of each tile
+    regs_dec<kRegsConv>();
+    const int t = threadIdx.x;                           // meta: position t of each tile
+    const int i8 = lane >> 2, kq = lane & 3;             // codes: positions 32 warp + 8m + i8, quarter kq
+    const uint32_t kb_a = smem_u32(kb), vb_a = smem_u32(vb);
+    PosMeta<KIND> cur, nxt;
+    Quarter<BITS> fc[4], fn[4];
+    if (n > 0) {
+      cur.load(a, b, kv, tile0 * kN + t, ctx);
+      load_quarters<BITS>(a, b, kv, tile0 * kN + 32 * warp + i8, ctx, kq, fc);
+    }
+    int e_cur = kNoScale;                                // running value-scale exponent
+    bool ok = true;
     for (int i = 0; i < n; ++i) {
-      const int buf = i & 1;
-      bool ok = mbar_wait(&bars->full, i & 1, abort);
-      uint32_t wk[4 * BITS], wv[4 * BITS];
-      if (ok) {
-        load_code_row<BITS>(stage, t, wk);
-        load_code_row<BITS>(stage + kN * C::kCode, t, wv);
+      const int st = i % kStages;
+      if (i + 1 < n) {
+        nxt.load(a, b, kv, (tile0 + i + 1) * kN + t, ctx);
+        load_quarters<BITS>(a, b, kv, (tile0 + i + 1) * kN + 32 * warp + i8, ctx, kq, fn);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->cfree);
-      const int pos = (tile0 + i) * kN + t;
       float ks = 0.f, kz = 0.f, vs = 0.f, vz = 0.f;
-      bool valid = false;
-      if (pos < ctx) {
-        const long long row = a.rows.row(b, kv, pos);
-        if (row >= 0) {
-          valid = true;
-          uint32_t km, vm;
-          if (KIND == WUSHKV_QUEST_INT) {
-            km = __ldg(a.k_meta + row);
-            vm = __ldg(a.v_meta + row);
-          } else {
-            km = __ldg(reinterpret_cast<const uint32_t*>(a.k_meta) + row);
-            vm = __ldg(reinterpret_cast<const uint32_t*>(a.v_meta) + row);
-          }
-          meta_of<KIND>(km, BITS, ks, kz);
-          meta_of<KIND>(vm, BITS, vs, vz);
-        } else {
-          report(a.status, WUSHKV_STATUS_BAD_PAGE);
-        }
+      if (cur.valid) {
+        meta_of<KIND>(cur.km, BITS, ks, kz);
+        meta_of<KIND>(cur.vm, BITS, vs, vz);
       }
-      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-      if (i >= 2) ok = mbar_wait(&bars->kvfree[buf], ((i - 2) >> 1) & 1, abort) && ok;
-      float* mt = reinterpret_cast<float*>(meta + buf * C::kMetaBytes);
+      // the tile's largest value scale (scales are >= 0, so their bits order like them)
+      const uint32_t smax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(vs)));
+      const uint32_t vmask = __ballot_sync(0xffffffffu, cur.valid);
+      if (lane == 0) sclx[st * 4 + warp] = smax;
+      named_barrier(1, 32 * kConvWarps);
+      const float tmax = __uint_as_float(max(max(sclx[st * 4], sclx[st * 4 + 1]),
+                                             max(sclx[st * 4 + 2], sclx[st * 4 + 3])));
+      if (tmax > 0.f) {
+        int et = 0;
+        frexpf(tmax, &et);                               // tmax < 2^et
+        e_cur = max(e_cur, et);
+      }
+      if (i >= kStages) ok = mbar_wait(&bars->kvfree[st], ((i - kStages) / kStages) & 1, abort) && ok;
+      float* mt = meta + st * kMetaWords;
       mt[t] = ks;
       mt[kN + t] = kz;
-      mt[2 * kN + t] = vs;
+      mt[2 * kN + t] = vs * exp2i(-e_cur);
       mt[3 * kN + t] = vz;
-      if (lane == 0) reinterpret_cast<uint32_t*>(mt + 4 * kN)[warp] = vmask;
+      uint32_t* mw = reinterpret_cast<uint32_t*>(mt + 4 * kN);
+      if (lane == 0) mw[warp] = vmask;
+      if (t == 0) mw[4] = (uint32_t)e_cur;
       if (ok) {
-        if (!valid) {
+        // keys: matrix (8 positions x slots 8c .. 8c + 7) -> rows = positions;
+        // values: the same matrix transposed -> rows = slots, 8 positions per row
+        const uint32_t kst = kb_a + st * 2 * kHalfBytes, vst = vb_a + st * 2 * kHalfBytes;
+        const int mj = lane >> 3, mr = lane & 7;         // this lane's row address: matrix mj, row mr
 #pragma unroll
-          for (int q = 0; q < 4 * BITS; ++q) { wk[q] = 0u; wv[q] = 0u; }
+        for (int m = 0; m < 4; ++m) {
+          const int p0 = 32 * warp + 8 * m;              // first position of the group
+#pragma unroll
+          for (int cg = 0; cg < 4; ++cg) {
+            const int c = 4 * cg + mj;                   // chunk (8 slots) of this lane's row address
+            const uint32_t ka = kst + (c >> 3) * kHalfBytes + (p0 + mr) * 128 + (((c & 7) ^ mr) << 4);
+            const int nrow = 8 * c + mr;
+            const uint32_t va = vst + (p0 >> 6) * kHalfBytes + nrow * 128 + ((((p0 & 63) >> 3) ^ (nrow & 7)) << 4);
+            stmatrix_x4(ka, code_pair_f16<BITS>(fc[m].k, 4 * cg), code_pair_f16<BITS>(fc[m].k, 4 * cg + 1),
+                        code_pair_f16<BITS>(fc[m].k, 4 * cg + 2), code_pair_f16<BITS>(fc[m].k, 4 * cg + 3));
+            stmatrix_x4_trans(va, code_pair_f16<BITS>(fc[m].v, 4 * cg), code_pair_f16<BITS>(fc[m].v, 4 * cg + 1),
+                              code_pair_f16<BITS>(fc[m].v, 4 * cg + 2), code_pair_f16<BITS>(fc[m].v, 4 * cg + 3));
+          }
         }
-        store_code_row<BITS>(kb + buf * 2 * kHalfBytes, t, wk);
-        store_code_row<BITS>(vb + buf * 2 * kHalfBytes, t, wv);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->conv[buf]);
+      if (lane == 0) mbar_arrive(&bars->conv[st]);
+      cur = nxt;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) fc[m] = fn[m];
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------- loads + MMAs
-    // The whole warp walks the tiles (the paged copies use several lanes); lane 0 waits
-    // and issues the MMAs, the other lanes follow it through __syncwarp.
+  } else if (warp >= kMmaWarp) {
+    // ------------------------------------------------------------- MMA issue
+    // The whole warp walks the tiles; lane 0 waits and issues, the others follow it.
+    regs_dec<kRegsMma>();
+    if (warp == kMmaWarp) {
     constexpr uint32_t kIdS = idesc(kFmtF32, kFmtF16, kFmtF16, 0, 0, 128, 128);
-    constexpr uint32_t kIdPV = idesc(kFmtF32, kFmtF16, kFmtF16, 0, 1, 128, 128);
-    const uint32_t qh_a = smem_u32(qh), ql_a = smem_u32(ql), kb_a = smem_u32(kb), vb_a = smem_u32(vb);
-    bool ok = true;
+    constexpr uint32_t kIdPV = idesc(kFmtF32, kFmtF16, kFmtF16, 0, 0, 128, 128);
+    const uint32_t kb_a = smem_u32(kb), vb_a = smem_u32(vb);
+    bool ok = true, issued = false;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       bool w = true;
       if (lane == 0) w = mbar_wait(bar, parity, abort);
@@ -370,114 +422,161 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!(ok = ok && wait_all(&bars->pfull, j & 1))) return;
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t vbase = vb_a + (j & 1) * 2 * kHalfBytes;
+        const uint32_t vbase = vb_a + (j % kStages) * 2 * kHalfBytes;
 #pragma unroll
         for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_f16_ts(tmem + kColO, tmem + kColP + pl * 64 + ks * 8,
-                       make_desc(vbase + ks * 2048, kHalfBytes, 1024, 2), kIdPV, (j > 0 || pl > 0 || ks > 0) ? 1u : 0u);
+          for (int k = 0; k < 8; ++k)
+            mma_f16_ts(tmem + kColO, tmem + kColP + pl * 64 + k * 8,
+                       desc_kmajor_sw128(vbase + (k >> 2) * kHalfBytes + (k & 3) * 32), kIdPV,
+                       (j > 0 || pl > 0 || k > 0) ? 1u : 0u);
         mma_commit(&bars->pvdone);
-        mma_commit(&bars->kvfree[j & 1]);
+        mma_commit(&bars->kvfree[j % kStages]);
+        issued = true;
       }
       __syncwarp();
     };
     for (int i = 0; i < n && ok; ++i) {
-      const int buf = i & 1;
-      if (i + 1 < n) {                                   // the next tile's codes, once these are read
-        if (!(ok = wait_all(&bars->cfree, i & 1))) break;
-        issue_load(i + 1);
-      }
-      if (!(ok = wait_all(&bars->conv[buf], (i >> 1) & 1))) break;
-      if (i >= 2 && !(ok = wait_all(&bars->sfree[buf], ((i - 2) >> 1) & 1))) break;
+      const int st = i % kStages;
+      if (!(ok = wait_all(&bars->conv[st], (i / kStages) & 1))) break;
+      if (i >= 1 && !(ok = wait_all(&bars->sfree, (i - 1) & 1))) break;
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t kbase = kb_a + buf * 2 * kHalfBytes;
+        const uint32_t kbase = kb_a + st * 2 * kHalfBytes;
 #pragma unroll
         for (int pl = 0; pl < 2; ++pl)
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-            mma_f16_ss(tmem + kColS + buf * 128, desc_kmajor_sw128((pl ? ql_a : qh_a) + off),
-                       desc_kmajor_sw128(kbase + off), kIdS, (pl | ks) != 0);
-          }
-        mma_commit(&bars->sfull[buf]);
+          for (int k = 0; k < 8; ++k)
+            mma_f16_ts(tmem + kColS, tmem + kColQ + pl * 64 + k * 8,
+                       desc_kmajor_sw128(kbase + (k >> 2) * kHalfBytes + (k & 3) * 32), kIdS, (pl | k) != 0);
+        mma_commit(&bars->sfull);
+        issued = true;
       }
       __syncwarp();
       if (i >= 1) pv(i - 1);
     }
     if (ok && n > 0) pv(n - 1);
-    // no copy may land after the CTA has exited, even after a timeout
-    if (lane == 0 && !ok && issued > 0) {
+    // no MMA may still run when the tensor memory is released, even after a timeout
+    if (lane == 0 && issued && *abort) {
       volatile int no_abort = 0;
-      mbar_wait(&bars->full, (issued - 1) & 1, &no_abort);
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, &no_abort);
+    }
+    __syncwarp();
     }
   } else {
     // ------------------------------------------------------------- softmax
+    regs_inc<kRegsSoft>();
+    const uint64_t rowc2 = pk2(rowc, rowc);
+    const uint64_t qs2 = pk2(qs, qs);
+    // QuEST: zero = -c0 * scale, so s = scale * (rowc * raw - c0 * qs)
+    const float c0 = (float)(1 << (BITS - 1)) - 0.5f;
+    const uint64_t cq2 = pk2(-c0 * qs, -c0 * qs);
     float m_ref = -CUDART_INF_F, l = 0.f, z = 0.f;
+    int e_prev = kNoScale;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
-      const int buf = i & 1;
-      ok = ok && mbar_wait(&bars->sfull[buf], (i >> 1) & 1, abort);
-      ok = ok && mbar_wait(&bars->conv[buf], (i >> 1) & 1, abort);
+      const int st = i % kStages;
+      ok = ok && mbar_wait(&bars->sfull, i & 1, abort);
+      ok = ok && mbar_wait(&bars->conv[st], (i / kStages) & 1, abort);
       tc_fence_after();
-      const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
       uint32_t raw[64];
-      tmem_ld32(tmem + lanes + kColS + buf * 128 + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(raw));
-      tmem_ld32(tmem + lanes + kColS + buf * 128 + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+      tmem_ld32(tmem + lanes + kColS + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(raw));
+      tmem_ld32(tmem + lanes + kColS + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->sfree[buf]);
-      const float* mt = reinterpret_cast<const float*>(meta + buf * C::kMetaBytes);
-      const uint32_t vm0 = reinterpret_cast<const uint32_t*>(mt + 4 * kN)[2 * hf];
-      const uint32_t vm1 = reinterpret_cast<const uint32_t*>(mt + 4 * kN)[2 * hf + 1];
+      if (lane == 0) mbar_arrive(&bars->sfree);
+      const float* mt = meta + st * kMetaWords;
+      const uint32_t* mw = reinterpret_cast<const uint32_t*>(mt + 4 * kN);
+      const uint32_t vm0 = mw[2 * hf], vm1 = mw[2 * hf + 1];
+      const int e_t = (int)mw[4];
       const int pos0 = (tile0 + i) * kN + 64 * hf;
-      float s[64];
-      float mloc = -CUDART_INF_F;
+      // x = s - base, base = the reference (0 before the row has seen a position)
+      const float base = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+      const uint64_t nb2 = pk2(-base, -base);
+      float x[64];
 #pragma unroll
       for (int j = 0; j < 64; j += 4) {
         const float4 k4 = *reinterpret_cast<const float4*>(mt + 64 * hf + j);
-        const float4 z4 = *reinterpret_cast<const float4*>(mt + kN + 64 * hf + j);
-        const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, zz[4] = {z4.x, z4.y, z4.z, z4.w};
+        const uint64_t r01 = pk2(__uint_as_float(raw[j]), __uint_as_float(raw[j + 1]));
+        const uint64_t r23 = pk2(__uint_as_float(raw[j + 2]), __uint_as_float(raw[j + 3]));
+        uint64_t x01, x23;
+        if (KIND == WUSHKV_QUEST_INT) {
+          x01 = fma2_rn(pk2(k4.x, k4.y), fma2_rn(rowc2, r01, cq2), nb2);
+          x23 = fma2_rn(pk2(k4.z, k4.w), fma2_rn(rowc2, r23, cq2), nb2);
+        } else {
+          const float4 z4 = *reinterpret_cast<const float4*>(mt + kN + 64 * hf + j);
+          x01 = fma2_rn(mul2_rn(pk2(k4.x, k4.y), r01), rowc2, fma2_rn(pk2(z4.x, z4.y), qs2, nb2));
+          x23 = fma2_rn(mul2_rn(pk2(k4.z, k4.w), r23), rowc2, fma2_rn(pk2(z4.z, z4.w), qs2, nb2));
+        }
+        unpk2(x01, x[j], x[j + 1]);
+        unpk2(x23, x[j + 2], x[j + 3]);
+      }
+      // causal mask and page validity, only where the tile reaches them
+      if (!(__all_sync(0xffffffffu, pos0 + 63 <= p_last) && (vm0 & vm1) == 0xffffffffu)) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int jj = j + e;
-          const bool vis = (((jj < 32 ? vm0 >> jj : vm1 >> (jj - 32)) & 1u) != 0u) && pos0 + jj <= p_last;
-          const float x = fmaf(kk[e] * rowc, __uint_as_float(raw[jj]), zz[e] * qs);
-          s[jj] = vis ? x : -CUDART_INF_F;
-          mloc = fmaxf(mloc, s[jj]);
+        for (int j = 0; j < 64; ++j) {
+          const bool vis = (((j < 32 ? vm0 >> j : vm1 >> (j - 32)) & 1u) != 0u) && pos0 + j <= p_last;
+          x[j] = vis ? x[j] : -CUDART_INF_F;
         }
       }
-      // tile maximum of the row (both halves)
+      float mloc = -CUDART_INF_F;
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) mloc = max3f(mloc, x[j], x[j + 1]);
+      // tile maximum of the row (both halves), relative to base
       rowx[4 * kRows + (i & 1) * 2 * kRows + hf * kRows + r] = mloc;
       named_barrier(bar_pair, 64);
-      const float m_tile = fmaxf(mloc, rowx[4 * kRows + (i & 1) * 2 * kRows + (1 - hf) * kRows + r]);
-      float m_new = m_ref;
-      if (m_tile != -CUDART_INF_F && (m_ref == -CUDART_INF_F || m_tile > m_ref + kLazy)) m_new = m_tile;
-      const bool rescale = m_new != m_ref && m_ref != -CUDART_INF_F;
-      const float corr = rescale ? ex2_approx(m_ref - m_new) : 1.f;
-      const float mref = m_new == -CUDART_INF_F ? 0.f : m_new;
-      // P' and O are free once the previous tile's PV MMA is done; O is rescaled when the
-      // reference moved
+      const float m_t = fmaxf(mloc, rowx[4 * kRows + (i & 1) * 2 * kRows + (1 - hf) * kRows + r]);
+      float shift = 0.f, corr = 1.f;
+      if (m_t != -CUDART_INF_F) {
+        if (m_ref == -CUDART_INF_F) {
+          shift = m_t;
+          m_ref = m_t;
+        } else if (m_t > kLazy) {
+          shift = m_t;
+          corr = ex2_approx(-m_t);
+          m_ref += m_t;
+        }
+      }
+      if (__any_sync(0xffffffffu, shift != 0.f)) {
+        const uint64_t s2 = pk2(-shift, -shift);
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+          uint64_t v2 = pk2(x[j], x[j + 1]);
+          v2 = add2_rn(v2, s2);
+          unpk2(v2, x[j], x[j + 1]);
+        }
+      }
+      // O carries the value scales times 2^-E: it grows by an exact power of two with E
+      const float corr_o = corr * (e_t > e_prev && i > 0 ? exp2i(max(e_prev - e_t, -126)) : 1.f);
+      e_prev = e_t;
+      // P' and O are free once the previous tile's PV MMAs are done
       if (i >= 1) ok = mbar_wait(&bars->pvdone, (i - 1) & 1, abort) && ok;
       tc_fence_after();
       // tensor-memory loads and stores are warp-collective: the warp rescales when any
-      // of its rows moved its reference (corr = 1 for the others)
+      // of its rows needs it (factor 1 for the others)
       ok = __all_sync(0xffffffffu, ok);
-      if (__any_sync(0xffffffffu, rescale) && ok) {
+      if (i > 0 && __any_sync(0xffffffffu, corr_o != 1.f) && ok) {
+        const uint64_t c2 = pk2(corr_o, corr_o);
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 16) {
+        for (int c0i = 0; c0i < 64; c0i += 16) {
           uint32_t ov[16];
-          tmem_ld16(tmem + lanes + kColO + 64 * hf + c0, ov);
+          tmem_ld16(tmem + lanes + kColO + 64 * hf + c0i, ov);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * corr);
-          tmem_st16(tmem + lanes + kColO + 64 * hf + c0, ov);
+          for (int e = 0; e < 16; e += 2) {
+            const uint64_t o2 = mul2_rn(pk2(__uint_as_float(ov[e]), __uint_as_float(ov[e + 1])), c2);
+            float o0, o1;
+            unpk2(o2, o0, o1);
+            ov[e] = __float_as_uint(o0);
+            ov[e + 1] = __float_as_uint(o1);
+          }
+          tmem_st16(tmem + lanes + kColO + 64 * hf + c0i, ov);
         }
       }
-      // P' = e * scale in fp16 hi + lo, 32 positions at a time
-      float lt = 0.f, zt = 0.f;
+      // e = 2^x; l, z; P' = e * scale * 2^-E in fp16 hi + lo, 32 positions at a time
+      uint64_t la = pk2(0.f, 0.f), lb = la, za = la, zb = la;
 #pragma unroll
       for (int jc = 0; jc < 64; jc += 32) {
         uint32_t ph[16], plo[16];
@@ -485,43 +584,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = jc; j < jc + 32; j += 4) {
           const float4 v4 = *reinterpret_cast<const float4*>(mt + 2 * kN + 64 * hf + j);
           const float4 w4 = *reinterpret_cast<const float4*>(mt + 3 * kN + 64 * hf + j);
-          const float vv[4] = {v4.x, v4.y, v4.z, v4.w}, ww[4] = {w4.x, w4.y, w4.z, w4.w};
-          float pp[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float ex = ex2_approx(s[j + e] - mref);
-            lt += ex;
-            zt = fmaf(ex, ww[e], zt);
-            pp[e] = ex * vv[e];
-          }
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const __half2 h2 = __floats2half2_rn(pp[e], pp[e + 1]);
-            const float2 hb = __half22float2(h2);
-            const __half2 l2 = __floats2half2_rn(pp[e] - hb.x, pp[e + 1] - hb.y);
-            ph[(j - jc + e) >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
-            plo[(j - jc + e) >> 1] = *reinterpret_cast<const uint32_t*>(&l2);
-          }
+          const uint64_t e01 = pk2(ex2_approx(x[j]), ex2_approx(x[j + 1]));
+          const uint64_t e23 = pk2(ex2_approx(x[j + 2]), ex2_approx(x[j + 3]));
+          la = add2_rn(la, e01);
+          lb = add2_rn(lb, e23);
+          za = fma2_rn(e01, pk2(w4.x, w4.y), za);
+          zb = fma2_rn(e23, pk2(w4.z, w4.w), zb);
+          const uint64_t p01 = mul2_rn(e01, pk2(v4.x, v4.y));
+          const uint64_t p23 = mul2_rn(e23, pk2(v4.z, v4.w));
+          float p0, p1, p2, p3;
+          unpk2(p01, p0, p1);
+          unpk2(p23, p2, p3);
+          const __half2 h01 = __floats2half2_rn(p0, p1), h23 = __floats2half2_rn(p2, p3);
+          const float2 b01 = __half22float2(h01), b23 = __half22float2(h23);
+          float d0, d1, d2, d3;
+          unpk2(sub2_rn(p01, pk2(b01.x, b01.y)), d0, d1);
+          unpk2(sub2_rn(p23, pk2(b23.x, b23.y)), d2, d3);
+          const __half2 l01 = __floats2half2_rn(d0, d1), l23 = __floats2half2_rn(d2, d3);
+          ph[(j - jc) >> 1] = *reinterpret_cast<const uint32_t*>(&h01);
+          ph[((j - jc) >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+          plo[(j - jc) >> 1] = *reinterpret_cast<const uint32_t*>(&l01);
+          plo[((j - jc) >> 1) + 1] = *reinterpret_cast<const uint32_t*>(&l23);
         }
         tmem_st16(tmem + lanes + kColP + 32 * hf + jc / 2, ph);
         tmem_st16(tmem + lanes + kColP + 64 + 32 * hf + jc / 2, plo);
       }
-      l = fmaf(l, corr, lt);
-      z = fmaf(z, corr, zt);
+      float l0, l1, l2, l3, z0, z1, z2, z3;
+      unpk2(la, l0, l1);
+      unpk2(lb, l2, l3);
+      unpk2(za, z0, z1);
+      unpk2(zb, z2, z3);
+      l = fmaf(l, corr, (l0 + l1) + (l2 + l3));
+      z = fmaf(z, corr, (z0 + z1) + (z2 + z3));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pfull);
-      m_ref = m_new;
     }
-    // ---- split partial of the row: m (log2 domain), l, o + z
+    // ---- split partial of the row: m (log2 domain), l, O 2^E + z
     uint32_t o[64];
 #pragma unroll
     for (int e = 0; e < 64; ++e) o[e] = 0u;
     if (n > 0) {
       ok = ok && mbar_wait(&bars->pvdone, (n - 1) & 1, abort);
       tc_fence_after();
-      const uint32_t lanes = (uint32_t)(32 * (warp & 3)) << 16;
       tmem_ld32(tmem + lanes + kColO + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(o));
       tmem_ld32(tmem + lanes + kColO + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
       tmem_ld_wait();
@@ -532,10 +638,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_barrier(bar_pair, 64);
     const float l_tot = l + rowx[(1 - hf) * kRows + r];
     const float z_tot = z + rowx[2 * kRows + (1 - hf) * kRows + r];
+    const float oscale = exp2i(min(max(e_prev, -126), 127));
     if (row_ok) {
       float* dst = a.ws + ((((size_t)b * a.n_q + qi) * a.hq + qh_idx) * a.num_splits + split) * kPartialStride;
 #pragma unroll
-      for (int e = 0; e < 64; ++e) dst[4 + slot_channel<BITS>(64 * hf + e)] = __uint_as_float(o[e]) + z_tot;
+      for (int e = 0; e < 64; ++e)
+        dst[4 + slot_channel<BITS>(64 * hf + e)] = fmaf(__uint_as_float(o[e]), oscale, z_tot);
       if (hf == 0) {
         dst[0] = m_ref;
         dst[1] = l_tot;
@@ -552,39 +660,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Tensor map over one side's codes ([planes][rows][16 * BITS bytes], boxes of box_rows rows,
-// swizzled as stage_swizzle reads them).
-template <int BITS>
-bool chunk_code_map(CUtensorMap* m, const uint8_t* base, int rows, int planes, int box_rows) {
-  const uint64_t dims[3] = {(uint64_t)(16 * BITS), (uint64_t)rows, (uint64_t)planes};
-  const uint64_t strides[2] = {(uint64_t)(16 * BITS), (uint64_t)rows * (16 * BITS)};
-  const uint32_t box[3] = {(uint32_t)(16 * BITS), (uint32_t)box_rows, 1};
-  const CUtensorMapSwizzle sw = BITS == 2 ? CU_TENSOR_MAP_SWIZZLE_32B
-                                : BITS == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                            : CU_TENSOR_MAP_SWIZZLE_NONE;
-  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box, sw);
-}
-
 template <int BITS>
 cudaError_t launch_bits(const wushkv_cache& c, const FaArgs& a, int batch, cudaStream_t stream) {
-  CUtensorMap km, vm;
-  const bool paged = c.block_table != nullptr;
-  const int rows = paged ? c.page_size : c.capacity;
-  const int planes = paged ? c.num_pages * c.num_kv_heads : c.batch * c.num_kv_heads;
-  if (!chunk_code_map<BITS>(&km, c.k_codes, rows, planes, a.box_rows) ||
-      !chunk_code_map<BITS>(&vm, c.v_codes, rows, planes, a.box_rows))
-    return cudaErrorInvalidValue;
   const dim3 grid(a.num_splits, a.hkv * a.row_blocks, batch);
   if (c.qp.kind == WUSHKV_QUEST_INT) {
     auto kern = chunk_fa_kernel<BITS, WUSHKV_QUEST_INT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FaCfg<BITS>::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, FaCfg<BITS>::kSmem, stream>>>(km, vm, a);
+    kern<<<grid, kThreads, kSmem, stream>>>(a);
   } else {
     auto kern = chunk_fa_kernel<BITS, WUSHKV_PCT_AFFINE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FaCfg<BITS>::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, FaCfg<BITS>::kSmem, stream>>>(km, vm, a);
+    kern<<<grid, kThreads, kSmem, stream>>>(a);
   }
   return cudaGetLastError();
 }
@@ -618,6 +706,8 @@ cudaError_t launch_chunk_attention(const wushkv_cache& c, const float* q_t, int 
                                    const int32_t* ctx_len, float softmax_scale, float* out, void* workspace,
                                    int num_splits, int32_t* status, cudaStream_t stream) {
   FaArgs a{};
+  a.k_codes = c.k_codes;
+  a.v_codes = c.v_codes;
   a.k_meta = c.k_meta;
   a.v_meta = c.v_meta;
   a.rows = CacheRows::of(c);
@@ -631,7 +721,6 @@ cudaError_t launch_chunk_attention(const wushkv_cache& c, const float* q_t, int 
   a.capacity = c.capacity;
   a.num_splits = num_splits > 0 ? num_splits : auto_chunk_splits(c, num_q_heads, n_q);
   a.row_blocks = row_blocks_of(n_q, num_q_heads / c.num_kv_heads);
-  a.box_rows = c.block_table != nullptr ? (c.page_size < kN ? c.page_size : kN) : kN;
   a.scale_log2 = softmax_scale * kLog2e;
   cudaError_t e;
   switch (c.qp.bits) {

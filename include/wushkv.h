@@ -297,11 +297,12 @@ WUSHKV_API size_t wushkv_chunk_workspace_bytes(const wushkv_cache* cache, int32_
  *                > capacity are clamped (WUSHKV_STATUS_CTX_OVERFLOW).
  *   out        : fp32 [batch][n_q][num_q_heads][128]; may not alias q_t.
  *   workspace  : at least wushkv_chunk_workspace_bytes() bytes, 16-byte aligned.
- *   num_splits : splits of the prefix (positions before the chunk); 0 = automatic.
- * The positions before the chunk run through the decode kernel with the chunk's
- * queries folded into the head group (at most 16 rows per KV head per pass, so
- * ceil(n_q * g / 16) passes over the prefix); the chunk's own positions take a
- * small causal kernel that also merges the two.  Errors as wushkv_decode_attention. */
+ *   num_splits : splits of the cached positions (1 .. 4096); 0 = automatic.
+ * The chunk's queries are folded into the head group (row i * g + h) and run on the
+ * tensor cores 128 rows at a time, so the cache is read once per (sequence, KV head)
+ * and block of 128 rows; the workspace holds one fp32 partial (m, l, o) per row and
+ * split, merged by a second launch.  Results do not depend on num_splits beyond fp32
+ * rounding.  Errors as wushkv_decode_attention. */
 WUSHKV_API int wushkv_chunk_attention(const wushkv_cache* cache, const float* q_t, int32_t n_q,
                            int32_t num_q_heads, const int32_t* ctx_len, float softmax_scale, float* out,
                            void* workspace, size_t workspace_bytes, int32_t num_splits, int32_t* status,
