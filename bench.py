@@ -42,7 +42,7 @@ L2_FLUSH_BYTES = 512 << 20
 # ncu summary of the decode kernel at this workload; its DRAM traffic is reported only
 # while the kernel sources still hash to the value recorded beside it.
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_tc_qwen8b_affine2.md")
-DECODE_SOURCES = ("decode_tc.cu", "sm100.cuh", "wushkv_common.cuh", "tmap.cu", "tmap.h")
+DECODE_SOURCES = ("decode_tc.cu", "sm100.cuh", "wushkv_common.cuh", "wushkv_quant.cuh", "tmap.cu", "tmap.h")
 APPEND_LAUNCHES, QUERY_LAUNCHES, DECODE_LAUNCHES = 1, 1, 2     # kernels per C-ABI call
 
 

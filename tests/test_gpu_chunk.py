@@ -92,6 +92,31 @@ def test_chunk_multi_tile_ctas(kind, bits, hq, hkv):
         assert ma <= MAX_ABS and rl <= REL_L2
 
 
+@pytest.mark.parametrize("kind,bits,v_scale", [(0, 2, (300.0, 3000.0)), (1, 4, (1e-3, 4e3))])
+def test_chunk_large_and_spread_value_scales(kind, bits, v_scale):
+    """Value scales far above 1 and spread over many binades: the kernel carries
+    e * scale in fp16, so it keeps the scales' running maximum exponent out of it."""
+    n_q, bsz, hq, hkv, cap = 16, 2, 8, 2, 700
+    c = gen.random_cache(bsz, hkv, cap, kind, bits, seed=41 + bits, device="cpu", v_scale_range=v_scale)
+    cache = dq.PackedCache(bsz, hkv, cap, kind, bits, tensors={k: v.cuda() for k, v in c.items()})
+    q = _chunk_queries(bsz, n_q, hq, seed=43).contiguous()
+    ctx = [700, 333]
+    cn = {name: t.numpy() for name, t in c.items()}
+    cn["k_meta"] = cn["k_meta"].view(np.uint16)
+    cn["v_meta"] = cn["v_meta"].view(np.uint16)
+    ref = orc.chunk_attention(cn, q.numpy().astype(np.float64), ctx, TAU, kind, bits, hkv)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = dq.chunk_attention(cache, q.cuda(), torch.tensor(ctx, dtype=torch.int32, device="cuda"), TAU,
+                             num_splits=1, status=st).cpu().numpy()
+    assert st.item() == 0
+    assert np.all(np.isfinite(got))
+    scale = float(np.abs(ref).max())
+    ma, rl = gu.attention_errors(got, ref)
+    print(f"kind={kind} bits={bits} v_scale={v_scale}: max|ref| {scale:.3g} max-abs {ma:.3e} rel-L2 {rl:.3e}")
+    # the bar scales with the values: 2e-3 of the largest output magnitude
+    assert ma <= MAX_ABS * max(1.0, scale) and rl <= REL_L2
+
+
 def test_chunk_last_query_and_splits():
     """The chunk's last query is the decode query at the same context; the split count
     changes results only at fp32 rounding level; contexts above the capacity are
