@@ -166,8 +166,8 @@ __device__ void quantize_group_warp(const float* x, const SmallArgs& a, bool sto
 // Key transform variants: none (keys given transformed), dense T_k, block-diagonal T_k
 // (blocks of tblock x tblock on the diagonal), and T_k = H diag(s) / sqrt(128).
 enum { kTfNone = 0, kTfDense = 1, kTfBlock = 2, kTfHadamard = 3 };
-static_assert(kTfDense == WUSHKV_TRANSFORM_DENSE && kTfBlock == WUSHKV_TRANSFORM_BLOCK_DIAG &&
-                  kTfHadamard == WUSHKV_TRANSFORM_HADAMARD_DIAG,
+static_assert((int)kTfDense == (int)WUSHKV_TRANSFORM_DENSE && (int)kTfBlock == (int)WUSHKV_TRANSFORM_BLOCK_DIAG &&
+                  (int)kTfHadamard == (int)WUSHKV_TRANSFORM_HADAMARD_DIAG,
               "transform kinds follow the C ABI");
 
 template <int BITS, int KIND, int TF, bool ROPE>
