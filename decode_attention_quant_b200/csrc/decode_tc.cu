@@ -732,9 +732,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<BITS, G>::kCtas)
 }
 
 // out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s   (log2-domain partials).
-// One pass over the splits in batches of eight whose loads are all in flight at once,
-// rescaling the running sums whenever a batch raises the maximum.
-constexpr int kCombineBatch = 8;
+// One pass over the splits in batches of sixteen whose loads are all in flight at once
+// (the automatic split counts of the workloads fit one or two batches), rescaling the
+// running sums whenever a batch raises the maximum.
+constexpr int kCombineBatch = 16;
 __global__ void __launch_bounds__(kHeadDim) combine_log2_kernel(const float* __restrict__ ws, int num_splits,
                                                                float* __restrict__ out) {
   const size_t bh = blockIdx.x;
