@@ -39,10 +39,10 @@ def _chunk_queries(bsz, n_q, hq, seed):
 
 @pytest.mark.parametrize("kind,bits,hq,hkv,n_q,ctx", [
     (0, 2, 4, 1, 16, [256]),               # tiny workload shape, one 16-token chunk at the end
-    (1, 2, 8, 2, 16, [300, 20]),           # g = 4: four passes of 16 folded rows
-    (0, 3, 16, 2, 16, [129, 7]),           # g = 8: eight passes; sequence 1 shorter than the chunk
-    (0, 4, 2, 2, 5, [260, 16]),            # g = 1, n_q = 5: one pass padded to 8 rows
-    (1, 4, 32, 2, 16, [1000, 513]),        # g = 16: sixteen passes
+    (1, 2, 8, 2, 16, [300, 20]),           # g = 4: 64 folded rows in one 128-row block
+    (0, 3, 16, 2, 16, [129, 7]),           # g = 8: one full row block; sequence 1 shorter than the chunk
+    (0, 4, 2, 2, 5, [260, 16]),            # g = 1, n_q = 5: 5 rows of a block
+    (1, 4, 32, 2, 16, [1000, 513]),        # g = 16: 256 folded rows, two row blocks
     (1, 3, 8, 2, 1, [77, 300]),            # n_q = 1: a decode query
 ])
 def test_chunk_matches_oracle(kind, bits, hq, hkv, n_q, ctx):
@@ -228,3 +228,50 @@ def test_chunk_after_gpu_append_end_to_end():
     ref = orc.chunk_attention(oc, qt_ref.reshape(1, n_q, hq, 128), [256], TAU, kind, bits, hkv)
     ma, rl = gu.attention_errors(got, ref)
     assert ma <= MAX_ABS and rl <= REL_L2, (ma, rl)
+
+
+def test_chunk_bad_page_entries():
+    """A block-table entry outside the pool: chunk attention leaves those positions out
+    (every query of the chunk) and raises the bad-page status bit."""
+    kind, bits, hq, hkv, bsz, cap, page, n_q = 1, 2, 8, 2, 2, 512, 128, 16
+    pps = cap // page
+    num_pages = bsz * pps
+    c = gen.random_cache(bsz, hkv, cap, kind, bits, seed=7, device="cuda")
+    bt = torch.randperm(num_pages, generator=torch.Generator().manual_seed(4))[:bsz * pps].view(bsz, pps)
+    bt = bt.to(torch.int32)
+    pools = {}
+    for name, t in c.items():
+        pool = torch.zeros((num_pages, hkv, page) + tuple(t.shape[3:]), dtype=t.dtype, device="cuda")
+        for b in range(bsz):
+            for p in range(pps):
+                pool[int(bt[b, p])] = t[b, :, p * page:(p + 1) * page]
+        pools[name] = pool
+    bad = bt.clone()
+    bad[1, 2] = num_pages                                   # positions 256..383 of sequence 1
+    paged = dq.PackedCache(bsz, hkv, cap, kind, bits, tensors=pools, page_size=page, num_pages=num_pages,
+                           block_table=bad)
+    q = _chunk_queries(bsz, n_q, hq, seed=9)
+    ctx = [512, 512]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = dq.chunk_attention(paged, q.cuda(), torch.tensor(ctx, dtype=torch.int32, device="cuda"), TAU,
+                             status=st).cpu().numpy()
+    torch.cuda.synchronize()
+    assert st.item() & dq.STATUS_BAD_PAGE
+    gsz = hq // hkv
+    worst = 0.0
+    for b in range(bsz):
+        for kv in range(hkv):
+            sel = {name: t[b, kv].cpu().numpy() for name, t in c.items()}
+            for i in range(n_q):
+                last = ctx[b] - n_q + i
+                keep = np.arange(last + 1)
+                if b == 1:
+                    keep = keep[(keep < 256) | (keep >= 384)]
+                ref = orc.decode_attention_pair(sel["k_codes"][keep], sel["k_meta"][keep].view(np.uint16),
+                                                sel["v_codes"][keep], sel["v_meta"][keep].view(np.uint16),
+                                                q[b, i, kv * gsz:(kv + 1) * gsz].numpy().astype(np.float64), TAU,
+                                                kind, bits)
+                ma, rl = gu.attention_errors(got[b, i, kv * gsz:(kv + 1) * gsz], ref)
+                worst = max(worst, ma)
+                assert ma <= MAX_ABS and rl <= REL_L2, (b, kv, i, ma, rl)
+    print(f"bad page: worst max-abs {worst:.3e}")
