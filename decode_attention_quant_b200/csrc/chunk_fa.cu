@@ -364,8 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_fa_kernel(const FaArgs a) {
                                              max(sclx[st * 4 + 2], sclx[st * 4 + 3])));
       if (tmax > 0.f) {
         int et = 0;
-        frexpf(tmax, &et);                               // tmax < 2^et
-        e_cur = max(e_cur, et);
+        frexpf(tmax, &et);                               // tmax < 2^et (fp16 scales: et <= 16)
+        e_cur = min(max(e_cur, et), 126);                // 2^-E stays a normal fp32
       }
       if (i >= kStages) ok = mbar_wait(&bars->kvfree[st], ((i - kStages) / kStages) & 1, abort) && ok;
       float* mt = meta + st * kMetaWords;
