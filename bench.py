@@ -405,7 +405,8 @@ def run_ours(args, rank, world, local):
                    "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
                    "head_dim": 128, "ctx": w.ctx, "quantizer": "percentile-affine 2-bit ranks 2/125",
                    "l2": "inputs larger than L2 (packed cache 302 MB > 126 MB L2)", "parallelism": f"replicas x{world}",
-                   "launch": "one CUDA graph of the timed steps" if graph is not None else "eager launches"},
+                   "launch": ("one CUDA graph of the timed steps" if graph is not None else "eager launches")
+                   + "; per step the query map runs on a side stream beside the append"},
         "step_bytes": step_bytes,
         "step_breakdown": breakdown,
         "roofline": {"bound": "hbm", "kernel": "decode call (split-K decode_tc_kernel + combine)",
