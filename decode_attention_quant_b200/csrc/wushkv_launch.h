@@ -37,7 +37,7 @@ cudaError_t launch_decode_attention(const wushkv_cache& c, const float* q_t, int
 // fp32 rows of 128: out[r] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
 cudaError_t launch_combine_partials(const float* ws, int rows, int num_splits, float* out, cudaStream_t stream);
 
-// Chunk attention (chunk.cu): workspace bytes and the call.
+// Chunk attention (chunk_fa.cu): workspace bytes and the call.
 size_t chunk_workspace_bytes(const wushkv_cache& c, int num_q_heads, int n_q, int num_splits);
 cudaError_t launch_chunk_attention(const wushkv_cache& c, const float* q_t, int n_q, int num_q_heads,
                                    const int32_t* ctx_len, float softmax_scale, float* out, void* workspace,
